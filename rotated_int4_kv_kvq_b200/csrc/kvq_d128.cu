@@ -1,0 +1,9 @@
+// Kernels and launchers for vectors of length d = 128.
+#include "kvq_inst.cuh"
+
+namespace kvq {
+template cudaError_t launch_fwd<128>(int, int, const FwdLaunch&);
+template cudaError_t launch_inv<128>(int, int, const InvLaunch&);
+template cudaError_t launch_decode<128>(int, int, const DecodeLaunch&);
+template cudaError_t read_status<128>(uint32_t*, bool);
+}  // namespace kvq

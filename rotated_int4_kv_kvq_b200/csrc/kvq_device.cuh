@@ -1,0 +1,369 @@
+// kvq_device.cuh -- device building blocks of libkvq (sm_100a).
+//
+// * PTX wrappers for mbarriers, TMA tensor copies and bulk-group waits.
+// * Compile-time twiddle factors (cos/sin of 2 pi k / n in double, rounded
+//   once to float) so that every FFT constant is an instruction immediate.
+// * Register-resident transforms: radix-2 decimation-in-frequency complex FFT
+//   (natural-order input, bit-reversed output slots, which are renamed at
+//   compile time) and the Walsh-Hadamard butterfly network.
+// * int4 quantize / pack and unpack / dequantize on 32-bit words.
+//
+// The method these pieces implement is described in include/kvq.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+namespace kvq {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kRotSRFT = 0;
+constexpr int kRotSRHT = 1;
+
+// 1.5 * 2^23: adding it to |t| < 2^22 rounds t to the nearest integer (ties
+// to even, the float32 default rounding) and leaves that integer, in two's
+// complement, in the low mantissa bits.
+constexpr float kRoundMagic = 12582912.0f;
+// 2^23 + 8: a float whose bits are 0x4B0000uu equals 2^23 + uu; subtracting
+// this gives uu - 8, i.e. the code of an offset-binary nibble uu = q + 8.
+constexpr float kUnpackMagic = 8388616.0f;
+
+// ------------------------------------------------------------ constexpr ---
+
+template <int B, int E, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (B < E) {
+    f(std::integral_constant<int, B>{});
+    static_for<B + 1, E>(f);
+  }
+}
+
+constexpr int ilog2(int n) {
+  int l = 0;
+  while ((1 << l) < n) ++l;
+  return l;
+}
+
+constexpr int bitrev(int x, int bits) {
+  int r = 0;
+  for (int i = 0; i < bits; ++i) r = (r << 1) | ((x >> i) & 1);
+  return r;
+}
+
+constexpr double kPi = 3.14159265358979323846264338327950288;
+
+// Taylor series, |x| <= pi/4: the first omitted term is below 1e-27.
+constexpr double taylor_sin(double x) {
+  double x2 = x * x, term = x, sum = x;
+  for (int n = 1; n < 13; ++n) {
+    term *= -x2 / double((2 * n) * (2 * n + 1));
+    sum += term;
+  }
+  return sum;
+}
+
+constexpr double taylor_cos(double x) {
+  double x2 = x * x, term = 1.0, sum = 1.0;
+  for (int n = 1; n < 13; ++n) {
+    term *= -x2 / double((2 * n - 1) * (2 * n));
+    sum += term;
+  }
+  return sum;
+}
+
+// cos(2 pi k / n), sin(2 pi k / n) with exact quadrant/octant reduction on
+// integers, so e.g. k/n = 1/4 gives exactly (0, 1).
+struct CS {
+  double c, s;
+};
+
+constexpr CS cos_sin_2pi(long k, long n) {
+  k %= n;
+  if (k < 0) k += n;
+  const long q = (4 * k) / n;  // quadrant
+  const long r = 4 * k - q * n;  // angle within quadrant = (pi/2) r / n
+  double c = 1.0, s = 0.0;
+  if (2 * r <= n) {
+    const double a = 0.5 * kPi * double(r) / double(n);
+    c = taylor_cos(a);
+    s = taylor_sin(a);
+  } else {
+    const double a = 0.5 * kPi * double(n - r) / double(n);
+    c = taylor_sin(a);
+    s = taylor_cos(a);
+  }
+  switch (q) {
+    case 0: return CS{c, s};
+    case 1: return CS{-s, c};
+    case 2: return CS{-c, -s};
+    default: return CS{s, -c};
+  }
+}
+
+constexpr float tw_cos(long k, long n) { return float(cos_sin_2pi(k, n).c); }
+constexpr float tw_sin(long k, long n) { return float(cos_sin_2pi(k, n).s); }
+
+constexpr double const_sqrt(double x) {  // Newton on a positive argument
+  double r = x > 1.0 ? x : 1.0;
+  for (int i = 0; i < 200; ++i) r = 0.5 * (r + x / r);
+  return r;
+}
+
+static_assert(tw_cos(1, 4) == 0.0f && tw_sin(1, 4) == 1.0f, "quarter turn");
+static_assert(tw_cos(1, 2) == -1.0f && tw_sin(1, 2) == 0.0f, "half turn");
+static_assert(cos_sin_2pi(1, 8).c - 0.70710678118654752 < 4e-16 &&
+                  cos_sin_2pi(1, 8).c - 0.70710678118654752 > -4e-16,
+              "eighth turn");
+static_assert(cos_sin_2pi(1, 6).c - 0.5 < 4e-16 && cos_sin_2pi(1, 6).c - 0.5 > -4e-16,
+              "sixth turn");
+static_assert(cos_sin_2pi(1, 12).s - 0.5 < 4e-16 && cos_sin_2pi(1, 12).s - 0.5 > -4e-16,
+              "twelfth turn");
+
+// ------------------------------------------------------------------ PTX ---
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after ~2 s (or 2^26
+// polls).  Returns false on time-out; callers record the error and stop.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 1023u) == 0 && global_timer_ns() - t0 > 2000000000ull) return false;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_1d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t x) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(x) : "memory");
+}
+
+// ------------------------------------------------------------- numerics ---
+
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t w) {
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ uint32_t float2_to_half2_bits(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // round to nearest even, both lanes
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// (dr + i di) * exp(-+ 2 pi i K / N), forward sign for INV = false.
+template <int N, int K, bool INV>
+__device__ __forceinline__ void twiddle(float dr, float di, float& outr, float& outi) {
+  if constexpr (K % N == 0) {
+    outr = dr;
+    outi = di;
+  } else if constexpr (4 * K == N) {
+    if constexpr (!INV) {  // * (-i)
+      outr = di;
+      outi = -dr;
+    } else {  // * (+i)
+      outr = -di;
+      outi = dr;
+    }
+  } else {
+    constexpr float c = tw_cos(K, N);
+    constexpr float s = tw_sin(K, N);
+    if constexpr (!INV) {  // * (c - i s)
+      outr = fmaf(dr, c, di * s);
+      outi = fmaf(di, c, -(dr * s));
+    } else {  // * (c + i s)
+      outr = fmaf(dr, c, -(di * s));
+      outi = fmaf(di, c, dr * s);
+    }
+  }
+}
+
+// In-place radix-2 DIF FFT of length N over (re, im) registers,
+// X_k = sum_n z_n exp(-+ 2 pi i k n / N) (no normalization).  Input in
+// natural order; X_k ends in slot bitrev(k).
+template <int N, bool INV>
+__device__ __forceinline__ void fft_dif(float (&re)[N], float (&im)[N]) {
+  constexpr int L = ilog2(N);
+  static_for<0, L>([&](auto st) {
+    constexpr int h = N >> (decltype(st)::value + 1);
+    static_for<0, N / 2>([&](auto b) {
+      constexpr int bb = decltype(b)::value;
+      constexpr int o = bb % h;
+      constexpr int i = (bb / h) * 2 * h + o;
+      constexpr int j = i + h;
+      const float ar = re[i], ai = im[i], br = re[j], bi = im[j];
+      re[i] = ar + br;
+      im[i] = ai + bi;
+      twiddle<2 * h, o, INV>(ar - br, ai - bi, re[j], im[j]);
+    });
+  });
+}
+
+// In-place unnormalized Walsh-Hadamard transform (Sylvester order).
+template <int N>
+__device__ __forceinline__ void fwht(float (&v)[N]) {
+  static_for<0, ilog2(N)>([&](auto st) {
+    constexpr int h = 1 << decltype(st)::value;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  });
+}
+
+// Max of |v[0..N)| as a balanced tree.
+template <int N>
+__device__ __forceinline__ float absmax(const float* v) {
+  if constexpr (N == 1) {
+    return fabsf(v[0]);
+  } else {
+    return fmaxf(absmax<N / 2>(v), absmax<N / 2>(v + N / 2));
+  }
+}
+
+// Eight round-to-int bit patterns (low byte = code) -> 8 packed nibbles:
+// byte j = (q_{2j} & 0xF) | (q_{2j+1} << 4).
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&f)[8]) {
+  const uint32_t e = __byte_perm(__byte_perm(f[0], f[2], 0x0040), __byte_perm(f[4], f[6], 0x0040),
+                                 0x5410);
+  const uint32_t o = __byte_perm(__byte_perm(f[1], f[3], 0x0040), __byte_perm(f[5], f[7], 0x0040),
+                                 0x5410);
+  return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+}
+
+// Codes of a packed word as exact floats q in [-8, 7], element order.
+__device__ __forceinline__ void unpack8(uint32_t w, float (&q)[8]) {
+  const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
+  const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    q[2 * j] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + j)) - kUnpackMagic;
+    q[2 * j + 1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + j)) - kUnpackMagic;
+  }
+}
+
+}  // namespace kvq

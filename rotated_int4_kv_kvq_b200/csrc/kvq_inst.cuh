@@ -1,0 +1,203 @@
+// kvq_inst.cuh -- host-side launchers for the kernels of one vector length d.
+// Included by exactly one translation unit per d (kvq_d64.cu, ...), which
+// explicitly instantiates launch_fwd<d>, launch_inv<d>, launch_decode<d> and
+// read_status<d>.
+#pragma once
+
+#include <algorithm>
+#include <mutex>
+
+#include "kvq_codec.cuh"
+#include "kvq_launch.h"
+
+namespace kvq {
+
+// Status word of this translation unit's kernels, one per device context.
+// Bit 0: a bounded wait on an asynchronous copy ran out.
+static __device__ unsigned g_status;
+
+template <int D>
+struct Tuning {
+  static constexpr int TPV = DefaultTPV<D>::value;
+  static constexpr int FWD_STAGES = D == 64 ? 3 : 2;
+  static constexpr int INV_STAGES = 3;
+};
+
+namespace detail {
+
+constexpr int kMaxDevices = 64;
+
+inline cudaError_t current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return e;
+  return (*dev >= 0 && *dev < kMaxDevices) ? cudaSuccess : cudaErrorInvalidDevice;
+}
+
+// Device address of g_status on the current device (looked up once).
+inline cudaError_t status_ptr(unsigned** out) {
+  static unsigned* ptrs[kMaxDevices];
+  static std::mutex mu;
+  int dev;
+  cudaError_t e = current_device(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = static_cast<unsigned*>(p);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
+// Opt the kernel into its dynamic shared memory and look up how many blocks
+// fit on one SM, once per kernel and device.
+template <auto Kern>
+cudaError_t setup(int smem, int* occ_out) {
+  static int occ[kMaxDevices];
+  static std::mutex mu;
+  int dev;
+  cudaError_t e = current_device(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  if (occ[dev] == 0) {
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int b = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, Kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    occ[dev] = std::max(b, 1);
+  }
+  *occ_out = occ[dev];
+  return cudaSuccess;
+}
+
+inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
+  const int64_t want = (n_tiles + kWarps - 1) / kWarps;
+  return int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count) * occ)));
+}
+
+template <int D, int G, int ROT>
+cudaError_t fwd_one(const FwdLaunch& L) {
+  using T = Tuning<D>;
+  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES>;
+  constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES>();
+  int occ;
+  unsigned* st;
+  cudaError_t e = setup<kern>(smem, &occ);
+  if (e == cudaSuccess) e = status_ptr(&st);
+  if (e != cudaSuccess) return e;
+  constexpr int vpw = 32 / T::TPV;
+  FwdArgs a{L.signs, L.scales, L.n_vec, (L.n_vec + vpw - 1) / vpw};
+  kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(*L.tmX, *L.tmQ, a, st);
+  return cudaGetLastError();
+}
+
+template <int D, int G, int ROT>
+cudaError_t inv_one(const InvLaunch& L) {
+  using T = Tuning<D>;
+  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES>;
+  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES>();
+  int occ;
+  unsigned* st;
+  cudaError_t e = setup<kern>(smem, &occ);
+  if (e == cudaSuccess) e = status_ptr(&st);
+  if (e != cudaSuccess) return e;
+  constexpr int vpw = 32 / T::TPV;
+  InvArgs a{L.signs, L.n_vec, (L.n_vec + vpw - 1) / vpw};
+  kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(*L.tmQ, *L.tmS,
+                                                                             *L.tmX, a, st);
+  return cudaGetLastError();
+}
+
+template <int D, int G, int ROT>
+cudaError_t decode_one(const DecodeLaunch& L) {
+  using T = Tuning<D>;
+  constexpr auto kern = kvq_decode_kernel<D, G, ROT, T::TPV, T::INV_STAGES>;
+  constexpr int smem = decode_smem_bytes<D, ROT, T::TPV, T::INV_STAGES>();
+  int occ;
+  unsigned* st;
+  cudaError_t e = setup<kern>(smem, &occ);
+  if (e == cudaSuccess) e = status_ptr(&st);
+  if (e != cudaSuccess) return e;
+  constexpr int vpw = 32 / T::TPV;
+  DecodeArgs a;
+  a.signs = L.signs;
+  a.scales = L.scales;
+  a.n_heads = L.n_heads;
+  a.cap = L.cap;
+  a.pos = L.pos;
+  a.n_new_tiles = (L.n_heads + vpw - 1) / vpw;
+  a.tok_tiles = (L.pos + vpw - 1) / vpw;
+  a.n_tiles = a.n_new_tiles + L.n_heads * a.tok_tiles;
+  kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(
+      *L.tmXn, *L.tmQn, *L.tmOn, *L.tmQc, *L.tmOc, a, st);
+  return cudaGetLastError();
+}
+
+// Run Op<D, G, ROT>(launch) for the runtime (group, rot) pair.
+template <int D, template <int, int, int> class Op, class L>
+cudaError_t dispatch(int group, int rot, const L& l) {
+  auto by_rot = [&](auto gc) -> cudaError_t {
+    constexpr int G = decltype(gc)::value;
+    if constexpr (G > D) {
+      return cudaErrorInvalidValue;
+    } else {
+      return rot == kRotSRFT ? Op<D, G, kRotSRFT>::run(l) : Op<D, G, kRotSRHT>::run(l);
+    }
+  };
+  switch (group) {
+    case 32: return by_rot(std::integral_constant<int, 32>{});
+    case 64: return by_rot(std::integral_constant<int, 64>{});
+    case 128: return by_rot(std::integral_constant<int, 128>{});
+    case 256: return by_rot(std::integral_constant<int, 256>{});
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D, int G, int ROT>
+struct FwdOp {
+  static cudaError_t run(const FwdLaunch& l) { return fwd_one<D, G, ROT>(l); }
+};
+template <int D, int G, int ROT>
+struct InvOp {
+  static cudaError_t run(const InvLaunch& l) { return inv_one<D, G, ROT>(l); }
+};
+template <int D, int G, int ROT>
+struct DecodeOp {
+  static cudaError_t run(const DecodeLaunch& l) { return decode_one<D, G, ROT>(l); }
+};
+
+}  // namespace detail
+
+template <int D>
+cudaError_t launch_fwd(int group, int rot, const FwdLaunch& L) {
+  return detail::dispatch<D, detail::FwdOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t launch_inv(int group, int rot, const InvLaunch& L) {
+  return detail::dispatch<D, detail::InvOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L) {
+  return detail::dispatch<D, detail::DecodeOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t read_status(uint32_t* value, bool clear) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (clear && v != 0) {
+    const unsigned z = 0;
+    e = cudaMemcpyToSymbol(g_status, &z, sizeof(z));
+    if (e != cudaSuccess) return e;
+  }
+  *value = v;
+  return cudaSuccess;
+}
+
+}  // namespace kvq

@@ -1,0 +1,62 @@
+// kvq_launch.h -- internal interface between the C-ABI front end (kvq_api.cu)
+// and the per-d kernel translation units (kvq_d64.cu, kvq_d128.cu,
+// kvq_d256.cu).  Not part of the public API.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvq {
+
+// Threads per vector and vectors per warp tile for each d (must match the
+// kernels' DefaultTPV).
+constexpr int tpv_of(int d) { return d >= 256 ? 2 : 1; }
+constexpr int vpw_of(int d) { return 32 / tpv_of(d); }
+
+struct FwdLaunch {
+  const CUtensorMap* tmX;  // x      [n_vec][d] fp16, box {64, VPW}, swizzle 128B
+  const CUtensorMap* tmQ;  // packed [n_vec][d/2] u8, box {d/2, VPW}, swizzle = pitch
+  const int8_t* signs;
+  float* scales;
+  int64_t n_vec;
+  int sm_count;
+  cudaStream_t stream;
+};
+
+struct InvLaunch {
+  const CUtensorMap* tmQ;  // packed, as above
+  const CUtensorMap* tmS;  // scales as 1-D f32, box {VPW * d/g}
+  const CUtensorMap* tmX;  // out, as x above
+  const int8_t* signs;
+  int64_t n_vec;
+  int sm_count;
+  cudaStream_t stream;
+};
+
+struct DecodeLaunch {
+  const CUtensorMap* tmXn;  // x_new [n_heads][d], box {64, VPW}
+  const CUtensorMap* tmQn;  // packed row pos of every head, box {d/2, VPW}
+  const CUtensorMap* tmOn;  // out row pos of every head, box {64, VPW}
+  const CUtensorMap* tmQc;  // packed cache 3-D {d/2, cap, n_heads}, box {d/2, VPW, 1}
+  const CUtensorMap* tmOc;  // out rows < pos 3-D {d, pos, n_heads}, box {64, VPW, 1}
+  const int8_t* signs;
+  float* scales;
+  int64_t n_heads, cap, pos;
+  int sm_count;
+  cudaStream_t stream;
+};
+
+// Implemented once per d in the matching translation unit.
+template <int D>
+cudaError_t launch_fwd(int group, int rot, const FwdLaunch& L);
+template <int D>
+cudaError_t launch_inv(int group, int rot, const InvLaunch& L);
+template <int D>
+cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L);
+// Reads (and optionally clears) the device status word of that translation
+// unit on the current device; the caller has synchronized the device.
+template <int D>
+cudaError_t read_status(uint32_t* value, bool clear);
+
+}  // namespace kvq

@@ -1,0 +1,157 @@
+"""Thin Python binding over the C ABI of libkvq.so (include/kvq.h).
+
+Argument marshalling only: tensors are checked and turned into raw device
+pointers; all work runs in the library's CUDA kernels.  PyTorch supplies the
+device memory and the stream.  There is no CPU fallback: importing this
+module fails if libkvq.so has not been built
+(``python -m rotated_int4_kv_kvq_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+SRFT = 0
+SRHT = 1
+
+KVQ_OK = 0
+STATUS = {
+    0: "KVQ_OK", 1: "KVQ_ERR_NULL", 2: "KVQ_ERR_BAD_DIM", 3: "KVQ_ERR_BAD_GROUP",
+    4: "KVQ_ERR_MISALIGNED", 5: "KVQ_ERR_BAD_ROT", 6: "KVQ_ERR_CUDA",
+    7: "KVQ_ERR_BAD_SIZE", 8: "KVQ_ERR_DEVICE_TIMEOUT", 9: "KVQ_ERR_UNSUPPORTED_DEVICE",
+}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
+
+EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_decode_step",
+           "kvq_status_string", "kvq_device_status", "kvq_version")
+
+
+class KVQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m rotated_int4_kv_kvq_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    lib.kvq_rot_quant_fwd.argtypes = [p, i64, i32, i32, p, i32, p, p, p]
+    lib.kvq_rot_quant_fwd.restype = i32
+    lib.kvq_dequant_rot_inv.argtypes = [p, p, i64, i32, i32, p, i32, p, p]
+    lib.kvq_dequant_rot_inv.restype = i32
+    lib.kvq_decode_step.argtypes = [p, p, p, i64, i64, i64, i32, i32, p, i32, p, p]
+    lib.kvq_decode_step.restype = i32
+    lib.kvq_status_string.argtypes = [i32]
+    lib.kvq_status_string.restype = ctypes.c_char_p
+    lib.kvq_device_status.argtypes = [i32]
+    lib.kvq_device_status.restype = i32
+    lib.kvq_version.argtypes = []
+    lib.kvq_version.restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.kvq_status_string(int(status)).decode()
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(fn: str, st: int):
+    if st != KVQ_OK:
+        raise KVQError(fn, st)
+
+
+def kvq_rot_quant_fwd(x: torch.Tensor, signs: torch.Tensor, rot: int, group: int,
+                      packed: torch.Tensor | None = None,
+                      scales: torch.Tensor | None = None, stream=None):
+    """Forward step on x [n_vec, d] fp16 -> (packed [n_vec, d/2] u8,
+    scales [n_vec, d/group] f32).  Outputs are allocated when not given."""
+    n, d = x.shape
+    _check(x, "x", torch.float16, (n, d))
+    _check(signs, "signs", torch.int8, (d,))
+    if packed is None:
+        packed = torch.empty((n, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, d // group), dtype=torch.float32, device=x.device)
+    _check(packed, "packed", torch.uint8, (n, d // 2))
+    _check(scales, "scales", torch.float32, (n, d // group))
+    st = lib.kvq_rot_quant_fwd(_ptr(x), n, d, group, _ptr(signs), rot, _ptr(packed),
+                               _ptr(scales), _stream(stream))
+    _raise("kvq_rot_quant_fwd", st)
+    return packed, scales
+
+
+def kvq_dequant_rot_inv(packed: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor,
+                        rot: int, group: int, out: torch.Tensor | None = None, stream=None):
+    """Inverse step -> out [n_vec, d] fp16 (allocated when not given)."""
+    n, half = packed.shape
+    d = 2 * half
+    _check(packed, "packed", torch.uint8, (n, half))
+    _check(scales, "scales", torch.float32, (n, d // group))
+    _check(signs, "signs", torch.int8, (d,))
+    if out is None:
+        out = torch.empty((n, d), dtype=torch.float16, device=packed.device)
+    _check(out, "out", torch.float16, (n, d))
+    st = lib.kvq_dequant_rot_inv(_ptr(packed), _ptr(scales), n, d, group, _ptr(signs), rot,
+                                 _ptr(out), _stream(stream))
+    _raise("kvq_dequant_rot_inv", st)
+    return out
+
+
+def kvq_decode_step(x_new: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, pos: int,
+                    signs: torch.Tensor, rot: int, group: int,
+                    out: torch.Tensor | None = None, stream=None):
+    """Decode step on a head-major cache: packed [H, cap, d/2] u8 and
+    scales [H, cap, d/group] f32 get row ``pos``; returns out [H, pos+1, d]."""
+    h, d = x_new.shape
+    cap = packed.shape[1]
+    _check(x_new, "x_new", torch.float16, (h, d))
+    _check(packed, "packed", torch.uint8, (h, cap, d // 2))
+    _check(scales, "scales", torch.float32, (h, cap, d // group))
+    _check(signs, "signs", torch.int8, (d,))
+    if out is None:
+        out = torch.empty((h, pos + 1, d), dtype=torch.float16, device=x_new.device)
+    _check(out, "out", torch.float16, (h, pos + 1, d))
+    st = lib.kvq_decode_step(_ptr(x_new), _ptr(packed), _ptr(scales), h, cap, pos, d, group,
+                             _ptr(signs), rot, _ptr(out), _stream(stream))
+    _raise("kvq_decode_step", st)
+    return out
+
+
+def kvq_device_status(clear: bool = True) -> int:
+    """Synchronize the device and return the kernels' device status code."""
+    return int(lib.kvq_device_status(1 if clear else 0))
+
+
+def kvq_version() -> int:
+    return int(lib.kvq_version())

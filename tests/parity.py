@@ -1,0 +1,94 @@
+"""Element-by-element comparison of the CUDA path with the CPU oracle.
+
+Tolerances (the codec's stated parity bar):
+* int4 codes: bit-exact, except codes whose oracle y/s lies within 1e-4 of a
+  rounding tie; such mismatches are counted, must be off by exactly one step,
+  and must stay below 1e-4 of all codes;
+* scales: 1e-6 relative (exactly 0 where the oracle's scale is 0);
+* x_hat: max-abs 2e-3 * max|x| (per vector), in fp32.  The inverse is checked
+  against the oracle's inverse of the GPU's own codes and scales, and end to
+  end against the oracle's x_hat for vectors with no near-tie code flip.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+import oracle.kvq_oracle as O
+
+TIE_WINDOW = 1e-4
+MAX_FLIP_FRACTION = 1e-4
+SCALE_RTOL = 1e-6
+XHAT_ATOL_REL = 2e-3
+
+
+@dataclass
+class Report:
+    n_codes: int
+    flips: int
+    max_scale_rel: float
+    max_inv_err: float
+    max_e2e_err: float
+
+    @property
+    def flip_fraction(self) -> float:
+        return self.flips / max(1, self.n_codes)
+
+
+def check_fwd(x16, signs, rot, group, packed, scales):
+    """Return (report-fields, flipped-row mask) for the forward step."""
+    x16 = np.asarray(x16, dtype=np.float16)
+    y = O.rotated_values(x16, signs, rot)
+    q_ref, s_ref = O.quantize_groups(y, group)
+    s = np.asarray(scales, dtype=np.float32)
+    q = O.unpack_nibbles(np.asarray(packed, dtype=np.uint8))
+    assert q.shape == q_ref.shape and s.shape == s_ref.shape
+
+    # scales
+    zero = s_ref == 0
+    assert np.all(s[zero] == 0), "scale of an all-zero group must be 0"
+    rel = np.abs(s.astype(np.float64) - s_ref) / np.where(zero, 1.0, s_ref)
+    max_rel = float(rel[~zero].max(initial=0.0))
+    assert max_rel <= SCALE_RTOL, f"scale rel err {max_rel:.3g}"
+
+    # codes
+    assert q.min(initial=0) >= -8 and q.max(initial=0) <= 7
+    diff = q.astype(np.int16) - q_ref.astype(np.int16)
+    bad = diff != 0
+    flips = int(bad.sum())
+    if flips:
+        dist = O.near_tie_distance(y, s_ref, group)
+        assert np.all(np.abs(diff[bad]) == 1), "a code differs by more than one step"
+        worst = float(dist[bad].max())
+        assert worst < TIE_WINDOW, f"code mismatch away from a tie (distance {worst:.3g})"
+        assert flips < MAX_FLIP_FRACTION * q.size, f"{flips} near-tie flips of {q.size}"
+    return q, s, flips, max_rel, bad.any(axis=1)
+
+
+def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None):
+    """x_hat of the GPU against the oracle inverse of the same codes/scales,
+    and against the oracle's own x_hat on rows without a code flip."""
+    x = np.asarray(x16, dtype=np.float16).astype(np.float64)
+    tol = XHAT_ATOL_REL * np.maximum(np.abs(x).max(axis=1, keepdims=True), 1e-30)
+    ref = O.dequant_rot_inv(packed, scales, signs, rot, group).astype(np.float64)
+    got = np.asarray(out, dtype=np.float16).astype(np.float64)
+    err = np.abs(got - ref)
+    inv_err = float((err / tol).max(initial=0.0))
+    assert np.all(err <= tol), f"inverse error {inv_err:.3g} x tolerance"
+    e2e = 0.0
+    p_ref, s_ref = O.rot_quant_fwd(np.asarray(x16, np.float16), signs, rot, group)
+    full = O.dequant_rot_inv(p_ref, s_ref, signs, rot, group).astype(np.float64)
+    rows = np.ones(x.shape[0], bool) if flipped_rows is None else ~flipped_rows
+    if rows.any():
+        e = np.abs(got[rows] - full[rows]) / tol[rows]
+        e2e = float(e.max())
+        assert e2e <= 1.0, f"end-to-end x_hat error {e2e:.3g} x tolerance"
+    return inv_err, e2e
+
+
+def full_check(x16, signs, rot, group, packed, scales, out) -> Report:
+    q, s, flips, max_rel, flipped = check_fwd(x16, signs, rot, group, packed, scales)
+    inv_err, e2e = check_inv(x16, signs, rot, group, packed, scales, out, flipped)
+    return Report(q.size, flips, max_rel, inv_err, e2e)

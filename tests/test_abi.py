@@ -1,0 +1,98 @@
+"""The C ABI of libkvq.so without a GPU: it loads, exports every function
+include/kvq.h declares, and rejects bad arguments on the host before any
+CUDA call (fake pointers below are never dereferenced)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from rotated_int4_kv_kvq_b200 import build
+    build.build()
+    from rotated_int4_kv_kvq_b200 import kvq as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_decode_step",
+               "kvq_status_string"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(kvq):
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for fn in declared_functions():
+        assert hasattr(lib, fn), fn
+    assert set(kvq.EXPORTS) == set(declared_functions())
+
+
+def test_status_strings(kvq):
+    for code in range(10):
+        assert kvq.status_string(code)
+    assert kvq.status_string(0) == "ok"
+    assert kvq.status_string(12345) == "unknown status"
+    assert kvq.kvq_version() >= 100
+
+
+A = 0x10000  # 16-byte aligned fake device address (never dereferenced)
+
+
+@pytest.mark.parametrize("d,g,rot,expect", [
+    (32, 32, 0, 2), (96, 32, 0, 2), (512, 32, 0, 2),
+    (64, 16, 0, 3), (64, 128, 0, 3), (128, 48, 1, 3), (256, 512, 1, 3),
+    (64, 32, 2, 5), (64, 32, -1, 5),
+])
+def test_bad_shape_is_rejected(kvq, d, g, rot, expect):
+    lib = kvq.lib
+    assert lib.kvq_rot_quant_fwd(A, 10, d, g, A, rot, A, A, None) == expect
+    assert lib.kvq_dequant_rot_inv(A, A, 10, d, g, A, rot, A, None) == expect
+    assert lib.kvq_decode_step(A, A, A, 2, 8, 3, d, g, A, rot, A, None) == expect
+
+
+def test_null_and_misaligned_pointers(kvq):
+    lib = kvq.lib
+    assert lib.kvq_rot_quant_fwd(None, 10, 64, 32, A, 0, A, A, None) == 1
+    assert lib.kvq_rot_quant_fwd(A, 10, 64, 32, None, 0, A, A, None) == 1
+    assert lib.kvq_rot_quant_fwd(A, 10, 64, 32, A, 0, A, None, None) == 1
+    assert lib.kvq_dequant_rot_inv(A, A, 10, 64, 32, A, 0, None, None) == 1
+    assert lib.kvq_decode_step(A, None, A, 2, 8, 3, 64, 32, A, 0, A, None) == 1
+    for bad in (A + 2, A + 8):
+        assert lib.kvq_rot_quant_fwd(bad, 10, 64, 32, A, 0, A, A, None) == 4
+        assert lib.kvq_rot_quant_fwd(A, 10, 64, 32, A, 0, bad, A, None) == 4
+        assert lib.kvq_rot_quant_fwd(A, 10, 64, 32, A, 0, A, bad, None) == 4
+        assert lib.kvq_dequant_rot_inv(A, A, 10, 64, 32, A, 0, bad, None) == 4
+        assert lib.kvq_decode_step(A, A, A, 2, 8, 3, 64, 32, A, 0, bad, None) == 4
+    assert lib.kvq_decode_step(A, A, A + 2, 2, 8, 3, 64, 32, A, 0, A, None) == 4
+
+
+def test_bad_sizes(kvq):
+    lib = kvq.lib
+    assert lib.kvq_rot_quant_fwd(A, -1, 64, 32, A, 0, A, A, None) == 7
+    assert lib.kvq_rot_quant_fwd(A, 1 << 31, 64, 32, A, 0, A, A, None) == 7
+    assert lib.kvq_dequant_rot_inv(A, A, -5, 64, 32, A, 0, A, None) == 7
+    # decode: pos must be < cap, cap >= 1, n_heads >= 0
+    assert lib.kvq_decode_step(A, A, A, 2, 8, 8, 64, 32, A, 0, A, None) == 7
+    assert lib.kvq_decode_step(A, A, A, 2, 0, 0, 64, 32, A, 0, A, None) == 7
+    assert lib.kvq_decode_step(A, A, A, -1, 8, 3, 64, 32, A, 0, A, None) == 7
+    assert lib.kvq_decode_step(A, A, A, 2, 8, -1, 64, 32, A, 0, A, None) == 7
+
+
+def test_empty_calls_are_noops(kvq):
+    lib = kvq.lib
+    assert lib.kvq_rot_quant_fwd(A, 0, 64, 32, A, 0, A, A, None) == 0
+    assert lib.kvq_dequant_rot_inv(A, A, 0, 256, 256, A, 1, A, None) == 0
+    assert lib.kvq_decode_step(A, A, A, 0, 8, 3, 128, 64, A, 0, A, None) == 0
