@@ -287,8 +287,18 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--suite", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run --reps forward+inverse passes of one shape (for ncu), no timing")
+    ap.add_argument("--rot", type=int, default=0)
+    ap.add_argument("--d", type=int, default=64)
+    ap.add_argument("--group", type=int, default=64)
+    ap.add_argument("--n-vec", type=int, default=1 << 21)
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.profile:
+        run_profile_case(args)
+        return
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, world, rank)
@@ -406,6 +416,31 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_profile_case(args):
+    """`reps` forward then inverse passes over n_vec vectors of the sweep
+    recipe at (d, group, rot): the small case ncu captures."""
+    from rotated_int4_kv_kvq_b200 import kvq
+    dev = torch.device("cuda", 0)
+    d, g = args.d, args.group
+    tokens = 8192
+    heads = max(1, -(-args.n_vec // (2 * tokens)))
+    shape = W.scaled(W.config(5, d=d, group=g), heads=heads, tokens=tokens)
+    x = W.make_kv(shape, device=dev)[: args.n_vec].contiguous()
+    signs = torch.from_numpy(W.make_signs(d)).to(dev)
+    packed, scales = kvq.kvq_rot_quant_fwd(x, signs, args.rot, g)
+    out = kvq.kvq_dequant_rot_inv(packed, scales, signs, args.rot, g)
+    for _ in range(args.reps):
+        kvq.kvq_rot_quant_fwd(x, signs, args.rot, g, packed, scales)
+        kvq.kvq_dequant_rot_inv(packed, scales, signs, args.rot, g, out)
+    torch.cuda.synchronize()
+    st = kvq.kvq_device_status()
+    print(json.dumps({"profile_case": {"d": d, "group": g, "rot": args.rot,
+                                       "n_vec": int(x.shape[0]), "reps": args.reps,
+                                       "status": st}}))
+    if st != 0:
+        sys.exit(1)
 
 
 def run_suite(kvq, dev):

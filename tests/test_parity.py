@@ -34,13 +34,13 @@ def run(kvq, x_dev, d, rot, group, signs_np):
     return packed, scales, out
 
 
-def check_all(kvq, x16, rot, group):
+def check_all(kvq, x16, rot, group, **kw):
     d = x16.shape[1]
     signs = W.make_signs(d)
     x_dev = torch.from_numpy(np.ascontiguousarray(x16)).cuda()
     p, s, o = run(kvq, x_dev, d, rot, group, signs)
     return full_check(x16, signs, rot, group, p.cpu().numpy(), s.cpu().numpy(),
-                      o.cpu().numpy())
+                      o.cpu().numpy(), **kw)
 
 
 @pytest.mark.parametrize("rot", ROTS)
@@ -88,7 +88,9 @@ def test_zero_and_extreme_vectors(kvq, d, rot):
     x[7, ::3] = 65504.0  # fp16 max
     x[8] = np.float16(6e-8)  # fp16 subnormals
     x[9, 0] = 1.0  # one-hot
-    rep = check_all(kvq, x, rot, 32)
+    # +-c vectors rotate onto exact ties, so near-tie flips are not capped;
+    # x_hat of +-60000 rows may overflow fp16 on both sides
+    rep = check_all(kvq, x, rot, 32, max_flip_fraction=None)
     signs = torch.from_numpy(W.make_signs(d)).cuda()
     p, s = kvq.kvq_rot_quant_fwd(torch.from_numpy(x).cuda(), signs, rot, 32)
     assert not s[0].any() and not p[0].any()
