@@ -27,6 +27,16 @@ namespace kvq {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 
+// Where a thread's E local rotated coordinates sit in the vector's y:
+//  kLayFull    (one thread per vector): local i is y[i].
+//  kLayHalf    (SRHT, thread pair):     thread t holds y[t*E + i].
+//  kLayQuarter (SRFT, thread pair):     local half h (E/2 values) of thread t is
+//           quarter qd = h ? 3 - 2t : 2t of y, i.e. thread 0 holds quarters
+//           0 and 3 and thread 1 quarters 2 and 1.  This is where the pair
+//           split of the real FFT leaves each output (see rotate_fwd), and it
+//           makes every (X_k, X_{N-k}) pair but one local to a thread.
+constexpr int kLayFull = 0, kLayHalf = 1, kLayQuarter = 2;
+
 template <int D_, int ROT_, int TPV_>
 struct Cfg {
   static constexpr int D = D_;
@@ -34,12 +44,14 @@ struct Cfg {
   static constexpr int TPV = TPV_;
   static constexpr int VPW = 32 / TPV;     // vectors per warp tile
   static constexpr int E = D / TPV;        // reals per thread
+  static constexpr int P = E / 2;          // float pairs per thread
   static constexpr int NW = E / 2;         // fp16-pair words per thread
   static constexpr int NQ = E / 8;         // packed-code words per thread
   static constexpr int XTILE = VPW * D * 2;  // fp16 tile bytes
   static constexpr int QTILE = VPW * D / 2;  // code tile bytes
   static constexpr int SLAB = VPW * 128;   // one 64-column fp16 slab
   static constexpr int QP = D / 2;         // code row pitch in bytes
+  static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
   // y = KAPPA * (unnormalized transform of u): SRFT 1/sqrt(2d), SRHT 1/sqrt(d)
   static constexpr double KAPPA_D =
       ROT == kRotSRFT ? 1.0 / const_sqrt(2.0 * D) : 1.0 / const_sqrt(double(D));
@@ -57,6 +69,21 @@ struct DefaultTPV {
 template <class C>
 __host__ __device__ constexpr int word_of(int t, int j) {
   return (C::ROT == kRotSRFT && C::TPV == 2) ? 2 * j + t : t * C::NW + j;
+}
+
+// Quarter of y holding local half h of thread t (kLayQuarter layout).
+__device__ __forceinline__ int quarter_of(int t, int h) { return h ? 3 - 2 * t : 2 * t; }
+
+// y index of local coordinate i of thread t.
+template <class C>
+__device__ __forceinline__ int global_y(int t, int i) {
+  if constexpr (C::LAYOUT == kLayFull) {
+    return i;
+  } else if constexpr (C::LAYOUT == kLayHalf) {
+    return t * C::E + i;
+  } else {
+    return quarter_of(t, i / (C::E / 2)) * (C::D / 4) + i % (C::E / 2);
+  }
 }
 
 template <class C>
@@ -135,11 +162,17 @@ __device__ __forceinline__ void store_x(uint32_t tile, int row, int t, uint32_t 
   }
 }
 
+// 16-byte code chunk of the row holding local code chunk lc of thread t.
+template <class C>
+__device__ __forceinline__ int code_chunk(int t, int lc) {
+  return global_y<C>(t, 32 * lc) / 32;
+}
+
 template <class C>
 __device__ __forceinline__ void load_codes(uint32_t tile, int row, int t, uint32_t (&qw)[C::NQ]) {
 #pragma unroll
   for (int c = 0; c < C::NQ / 4; ++c) {
-    const uint4 v = lds128(tile + swq<C::QP>(row, t * (C::NQ / 4) + c));
+    const uint4 v = lds128(tile + swq<C::QP>(row, code_chunk<C>(t, c)));
     qw[4 * c] = v.x;
     qw[4 * c + 1] = v.y;
     qw[4 * c + 2] = v.z;
@@ -152,117 +185,122 @@ __device__ __forceinline__ void store_codes(uint32_t tile, int row, int t,
                                             const uint32_t (&qw)[C::NQ]) {
 #pragma unroll
   for (int c = 0; c < C::NQ / 4; ++c)
-    sts128(tile + swq<C::QP>(row, t * (C::NQ / 4) + c), qw[4 * c], qw[4 * c + 1], qw[4 * c + 2],
+    sts128(tile + swq<C::QP>(row, code_chunk<C>(t, c)), qw[4 * c], qw[4 * c + 1], qw[4 * c + 2],
            qw[4 * c + 3]);
 }
 
 // ------------------------------------------------------ forward rotation ---
 
-// Y (this thread's E consecutive rotated coordinates, unnormalized: the true
-// y is KAPPA * Y) from the sign-flipped fp16 words.
+constexpr float kSqrt2 = 1.41421356237309504880f;
+
+// Y: this thread's E rotated coordinates as P pairs (local order of the
+// layout), unnormalized: the true y is KAPPA * Y.  Input: sign-flipped fp16
+// words.
 template <class C>
-__device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, float (&Y)[C::E]) {
+__device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f2 (&Y)[C::P]) {
   if constexpr (C::ROT == kRotSRHT) {
 #pragma unroll
     for (int j = 0; j < C::NW; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
-      Y[2 * j] = f.x;
-      Y[2 * j + 1] = f.y;
+      Y[j] = mk2(f.x, f.y);
     }
-    fwht<C::E>(Y);
+    fwht<C::P>(Y);
     if constexpr (C::TPV == 2) {  // H_d = [[H, H], [H, -H]] across the pair
       const float sg = t ? -1.0f : 1.0f;
+      const f2 sg2 = mk2(sg, sg);
 #pragma unroll
-      for (int i = 0; i < C::E; ++i) {
-        const float p = __shfl_xor_sync(kFull, Y[i], 1);
-        Y[i] = fmaf(sg, Y[i], p);
-      }
+      for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
     }
   } else if constexpr (C::TPV == 1) {
     // z_n = u_{2n} + i u_{2n+1}; Z = FFT_{d/2}(z); X_k from (Z_k, Z_{d/2-k}).
     constexpr int N = C::D / 2;
     constexpr int LN = ilog2(N);
-    float zr[N], zi[N];
+    f2 z[N];
 #pragma unroll
     for (int j = 0; j < N; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
-      zr[j] = f.x;
-      zi[j] = f.y;
+      z[j] = mk2(f.x, f.y);
     }
-    fft_dif<N, false>(zr, zi);
-    constexpr float R2 = 1.41421356237309504880f;
-    Y[0] = R2 * (zr[0] + zi[0]);  // sqrt2 * X_0
-    Y[1] = R2 * (zr[0] - zi[0]);  // sqrt2 * X_{d/2}
+    fft_dif<N, false>(z);
+    {
+      const float a = lo2(z[0]), b = hi2(z[0]);
+      Y[0] = mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));  // sqrt2 X_0, sqrt2 X_{d/2}
+    }
     static_for<1, N / 2>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
-      constexpr int sa = bitrev(k, LN), sb = bitrev(N - k, LN);
-      const float ar = zr[sa], ai = zi[sa], br = zr[sb], bi = -zi[sb];  // B = conj Z_{N-k}
-      const float sr = ar + br, si = ai + bi, tr = ar - br, ti = ai - bi;
-      // 2X_k = S + W^k (-i T), 2X_{N-k} = conj(S - W^k (-i T)), W = exp(-2 pi i / d)
+      // P1 = Z_k + Z_{N-k} = (Sr, Ti), P2 = Z_k - Z_{N-k} = (Tr, Si) where
+      // S = Z_k + conj Z_{N-k} = 2E_k and T = Z_k - conj Z_{N-k} = 2i O_k.
+      const f2 p1 = add2(z[bitrev(k, LN)], z[bitrev(N - k, LN)]);
+      const f2 p2 = sub2(z[bitrev(k, LN)], z[bitrev(N - k, LN)]);
+      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
+      // W^k (-i T), W = exp(-2 pi i / d)
       constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float pr = ti, pi = -tr;
-      const float wr = fmaf(c, pr, s * pi), wi = fmaf(c, pi, -(s * pr));
-      Y[2 * k] = sr + wr;
-      Y[2 * k + 1] = si + wi;
-      Y[2 * (N - k)] = sr - wr;
-      Y[2 * (N - k) + 1] = wi - si;
+      const float wr = fmaf(c, ti, -(s * tr)), wi = -fmaf(c, tr, s * ti);
+      Y[k] = mk2(sr + wr, si + wi);          // 2 X_k
+      Y[N - k] = mk2(sr - wr, wi - si);      // 2 X_{N-k} = conj(S - W^k (-i T))
     });
-    constexpr int sm = bitrev(N / 2, LN);
-    Y[N] = 2.0f * zr[sm];  // 2X_{d/4} = 2 conj Z_{d/4}
-    Y[N + 1] = -2.0f * zi[sm];
+    {
+      const f2 zm = z[bitrev(N / 2, LN)];
+      Y[N / 2] = mk2(2.0f * lo2(zm), -2.0f * hi2(zm));  // 2 X_{d/4} = 2 conj Z_{d/4}
+    }
   } else {
-    // TPV = 2.  Thread t holds z_{2m+t} (m < M = d/4): in-thread FFT_M, then
-    // the last decimation-in-time stage across the pair gives thread t the
-    // outputs Z_{k + t M}; X_k for those k uses the partner's Z_{d/2-k}.
+    // Thread pair, d/2 = N complex points, M = N/2 per thread, Q = M/2.
+    // Thread t holds z_{2m+t}: in-thread FFT_M gives F_t(k); thread 1 turns
+    // F_1(k) into G(k) = W_N^k F_1(k); one exchange gives, per slot k,
+    //   k <  Q: thread 0 Z_k = F0 + G,        thread 1 Z_{k+M} = F0 - G,
+    //   k >= Q: thread 0 Z_{k+M} = F0 - G,    thread 1 Z_k = F0 + G,
+    // so that both threads pair slot k with slot M - k for the real split
+    // (only the pair (Q, Q) straddles the threads).
     constexpr int M = C::D / 4;
     constexpr int N = C::D / 2;
+    constexpr int Q = M / 2;
     constexpr int LM = ilog2(M);
-    float zr[M], zi[M];
+    f2 z[M];
 #pragma unroll
     for (int j = 0; j < M; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
-      zr[j] = f.x;
-      zi[j] = f.y;
+      z[j] = mk2(f.x, f.y);
     }
-    fft_dif<M, false>(zr, zi);
+    fft_dif<M, false>(z);
     const float sg = t ? -1.0f : 1.0f;
+    const f2 sgA = mk2(sg, sg), sgB = mk2(-sg, -sg);
     static_for<0, M>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
       constexpr int sl = bitrev(k, LM);
-      float r = zr[sl], i = zi[sl];
+      f2 own = z[sl];
       if constexpr (k != 0) {
-        float wr, wi;
-        twiddle<N, k, false>(r, i, wr, wi);
-        r = t ? wr : r;
-        i = t ? wi : i;
+        if (t) own = twiddle<N, k, false>(own);
       }
-      const float pr = __shfl_xor_sync(kFull, r, 1);
-      const float pi = __shfl_xor_sync(kFull, i, 1);
-      zr[sl] = fmaf(sg, r, pr);  // t=0: F0 + W F1; t=1: F0 - W F1
-      zi[sl] = fmaf(sg, i, pi);
+      const f2 p = shfl_xor2(own, 1);
+      z[sl] = (k < Q) ? fma2(sgA, own, p) : fma2(sgB, p, own);
     });
-    constexpr float R2 = 1.41421356237309504880f;
-    {
-      const float a = zr[0], b = zi[0];
-      Y[0] = t ? 2.0f * a : R2 * (a + b);  // t=1 holds Z_{d/4}: 2 conj Z_{d/4}
-      Y[1] = t ? -2.0f * b : R2 * (a - b);
+    {  // slot 0: thread 0 Z_0 -> sqrt2 X_0, sqrt2 X_{d/2}; thread 1 Z_M -> 2 conj Z_M
+      const float a = lo2(z[0]), b = hi2(z[0]);
+      Y[0] = t ? mk2(2.0f * a, -2.0f * b) : mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
     }
-    static_for<1, M>([&](auto kk) {
+    static_for<1, Q>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
-      constexpr int sa = bitrev(k, LM), sb = bitrev(M - k, LM);
-      const float ar = zr[sa], ai = zi[sa];
-      const float br = __shfl_xor_sync(kFull, zr[sb], 1);
-      const float bi = -__shfl_xor_sync(kFull, zi[sb], 1);
-      const float sr = ar + br, si = ai + bi;
-      const float ur = br - ar, ui = bi - ai;  // U = -T
-      // thread 0: P = -i T = (-ui, ur); thread 1: W^{M} = -i folds in, P = -T = U
-      const float pr = t ? ur : -ui;
-      const float pi = t ? ui : ur;
+      const f2 p1 = add2(z[bitrev(k, LM)], z[bitrev(M - k, LM)]);
+      const f2 p2 = sub2(z[bitrev(k, LM)], z[bitrev(M - k, LM)]);
+      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
+      // thread 0: W_d^k (-i T); thread 1 holds Z_{k+M}: W_d^{k+M} = -i W_d^k,
+      // so it applies W_d^k to (-T).
+      const float pr = t ? -tr : ti, pi = t ? -ti : -tr;
       constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
       const float wr = fmaf(c, pr, s * pi), wi = fmaf(c, pi, -(s * pr));
-      Y[2 * k] = sr + wr;
-      Y[2 * k + 1] = si + wi;
+      Y[k] = mk2(sr + wr, si + wi);
+      Y[M - k] = mk2(sr - wr, wi - si);
     });
+    {  // slot Q: partner across the pair; thread 0 makes X_{Q+M}, thread 1 X_Q
+      const f2 own = z[bitrev(Q, LM)];
+      const f2 other = shfl_xor2(own, 1);
+      const f2 p1 = add2(own, other), p2 = sub2(own, other);
+      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
+      const float pr = t ? ti : -tr, pi = t ? -tr : -ti;
+      constexpr float c = tw_cos(Q, C::D), s = tw_sin(Q, C::D);
+      const float wr = fmaf(c, pr, s * pi), wi = fmaf(c, pi, -(s * pr));
+      Y[Q] = mk2(sr + wr, si + wi);
+    }
   }
 }
 
@@ -273,124 +311,166 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
 // inverse of rotate_fwd's unnormalized map up to the factor 1/KAPPA^2) yields
 // u itself.
 template <class C>
-__device__ __forceinline__ void rotate_inv(float (&Y)[C::E], int t, uint32_t (&xw)[C::NW]) {
+__device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[C::NW]) {
   if constexpr (C::ROT == kRotSRHT) {
     if constexpr (C::TPV == 2) {
       const float sg = t ? -1.0f : 1.0f;
+      const f2 sg2 = mk2(sg, sg);
 #pragma unroll
-      for (int i = 0; i < C::E; ++i) {
-        const float p = __shfl_xor_sync(kFull, Y[i], 1);
-        Y[i] = fmaf(sg, Y[i], p);
-      }
+      for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
     }
-    fwht<C::E>(Y);
+    fwht<C::P>(Y);
 #pragma unroll
-    for (int j = 0; j < C::NW; ++j) xw[j] = float2_to_half2_bits(Y[2 * j], Y[2 * j + 1]);
+    for (int j = 0; j < C::NW; ++j) xw[j] = float2_to_half2_bits(lo2(Y[j]), hi2(Y[j]));
   } else if constexpr (C::TPV == 1) {
     constexpr int N = C::D / 2;
     constexpr int LN = ilog2(N);
-    constexpr float R2 = 1.41421356237309504880f;
-    float zr[N], zi[N];
+    f2 z[N];
+    {
+      const float a = lo2(Y[0]), b = hi2(Y[0]);
+      z[0] = mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
+    }
     // Q_k = (A + B) + i W^{-k} (A - B), A = X'_k, B = conj X'_{N-k}
-    zr[0] = R2 * (Y[0] + Y[1]);
-    zi[0] = R2 * (Y[0] - Y[1]);
     static_for<1, N / 2>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
-      const float ar = Y[2 * k], ai = Y[2 * k + 1];
-      const float br = Y[2 * (N - k)], bi = -Y[2 * (N - k) + 1];
-      const float sr = ar + br, si = ai + bi, dr = ar - br, di = ai - bi;
+      const f2 p1 = add2(Y[k], Y[N - k]);  // (Sr, Di) with B = conj Y[N-k]
+      const f2 p2 = sub2(Y[k], Y[N - k]);  // (Dr, Si)
+      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
       constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
       const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);  // W^{-k} D
-      zr[k] = sr - vi;  // Q_k = S + i V
-      zi[k] = si + vr;
-      zr[N - k] = sr + vi;  // Q_{N-k} = conj(S - i V)
-      zi[N - k] = vr - si;
+      z[k] = mk2(sr - vi, si + vr);      // S + i V
+      z[N - k] = mk2(sr + vi, vr - si);  // conj(S - i V)
     });
-    zr[N / 2] = 2.0f * Y[N];
-    zi[N / 2] = -2.0f * Y[N + 1];
-    fft_dif<N, true>(zr, zi);
+    z[N / 2] = mk2(2.0f * lo2(Y[N / 2]), -2.0f * hi2(Y[N / 2]));
+    fft_dif<N, true>(z);
     static_for<0, N>([&](auto nn) {
       constexpr int n = decltype(nn)::value;
-      constexpr int sl = bitrev(n, LN);
-      xw[n] = float2_to_half2_bits(zr[sl], zi[sl]);
+      const f2 v = z[bitrev(n, LN)];
+      xw[n] = float2_to_half2_bits(lo2(v), hi2(v));
     });
   } else {
     constexpr int M = C::D / 4;
     constexpr int N = C::D / 2;
+    constexpr int Q = M / 2;
     constexpr int LM = ilog2(M);
-    constexpr float R2 = 1.41421356237309504880f;
-    float zr[M], zi[M];
+    f2 z[M];
     {
-      const float a = Y[0], b = Y[1];
-      zr[0] = t ? 2.0f * a : R2 * (a + b);
-      zi[0] = t ? -2.0f * b : R2 * (a - b);
+      const float a = lo2(Y[0]), b = hi2(Y[0]);
+      z[0] = t ? mk2(2.0f * a, -2.0f * b) : mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
     }
-    static_for<1, M>([&](auto kk) {
+    static_for<1, Q>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
-      const float ar = Y[2 * k], ai = Y[2 * k + 1];
-      const float br = __shfl_xor_sync(kFull, Y[2 * (M - k)], 1);
-      const float bi = -__shfl_xor_sync(kFull, Y[2 * (M - k) + 1], 1);
-      const float sr = ar + br, si = ai + bi, dr = ar - br, di = ai - bi;
+      const f2 p1 = add2(Y[k], Y[M - k]);
+      const f2 p2 = sub2(Y[k], Y[M - k]);
+      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
       constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);
-      // thread 0: Q = S + i V; thread 1: W^{-M} = +i folds in, Q = S - V
-      zr[k] = sr - (t ? vr : vi);
-      zi[k] = si + (t ? -vi : vr);
+      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);  // W_d^{-k} D
+      // thread 0: Q_k = S + i V, Q_{N-k} = conj(S - i V); thread 1 holds
+      // X'_{k+M}: W_d^{-(k+M)} = i W_d^{-k}, so Q = S - V, conj(S + V).
+      z[k] = t ? mk2(sr - vr, si - vi) : mk2(sr - vi, si + vr);
+      z[M - k] = t ? mk2(sr + vr, -(si + vi)) : mk2(sr + vi, vr - si);
     });
-    // Inverse of the cross-pair stage: thread 0 keeps E_k = Q_k + Q_{k+M},
-    // thread 1 keeps O_k = (Q_k - Q_{k+M}) W_{d/2}^{-k}.
+    {  // slot Q: thread 0 holds X'_{Q+M}, thread 1 X'_Q; partner across
+      const f2 other = shfl_xor2(Y[Q], 1);
+      const f2 p1 = add2(Y[Q], other), p2 = sub2(Y[Q], other);
+      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
+      constexpr float c = tw_cos(Q, C::D), s = tw_sin(Q, C::D);
+      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);
+      z[Q] = t ? mk2(sr - vi, si + vr) : mk2(sr - vr, si - vi);
+    }
+    // Inverse of the pair exchange: thread 0 forms E_k = Q_k + Q_{k+M},
+    // thread 1 O_k = (Q_k - Q_{k+M}) W_N^{-k}.
     const float sg = t ? -1.0f : 1.0f;
+    const f2 sgA = mk2(sg, sg);
     static_for<0, M>([&](auto kk) {
       constexpr int k = decltype(kk)::value;
-      const float pr = __shfl_xor_sync(kFull, zr[k], 1);
-      const float pi = __shfl_xor_sync(kFull, zi[k], 1);
-      float r = fmaf(sg, zr[k], pr), i = fmaf(sg, zi[k], pi);
+      const f2 own = z[k];
+      const f2 p = shfl_xor2(own, 1);
+      f2 r = (k < Q) ? fma2(sgA, own, p) : fma2(sgA, p, own);
       if constexpr (k != 0) {
-        float wr, wi;
-        twiddle<N, k, true>(r, i, wr, wi);
-        r = t ? wr : r;
-        i = t ? wi : i;
+        if (t) r = twiddle<N, k, true>(r);
       }
-      zr[k] = r;
-      zi[k] = i;
+      z[k] = r;
     });
-    fft_dif<M, true>(zr, zi);
+    fft_dif<M, true>(z);
     static_for<0, M>([&](auto mm) {
       constexpr int m = decltype(mm)::value;
-      constexpr int sl = bitrev(m, LM);
-      xw[m] = float2_to_half2_bits(zr[sl], zi[sl]);
+      const f2 v = z[bitrev(m, LM)];
+      xw[m] = float2_to_half2_bits(lo2(v), hi2(v));
     });
   }
 }
 
 // ------------------------------------------------------ quantize / pack ---
 
-template <class C, int G>
-struct Groups {
-  static constexpr int GL = G <= C::E ? G : C::E;  // group length in this thread
-  static constexpr int NL = C::E / GL;             // groups (scales) per thread
-  static constexpr bool SHARED = G > C::E;         // one group over the pair
-  static constexpr int NG = C::D / G;              // scales per vector
-  static_assert(GL % 8 == 0, "group");
-};
+constexpr int kXNone = 0, kXShared = 1, kXCrossHalf = 2, kXAll = 3;
 
 template <class C, int G>
-__device__ __forceinline__ void quantize(const float (&Y)[C::E], uint32_t (&qw)[C::NQ],
+struct Groups {
+  static constexpr int GL =
+      C::LAYOUT == kLayQuarter ? (G <= C::E / 2 ? G : C::E / 2) : (G <= C::E ? G : C::E);
+  static constexpr int NL = C::E / GL;  // local groups (scales) per thread
+  static constexpr int NG = C::D / G;   // scales per vector
+  static constexpr int X = C::LAYOUT == kLayFull    ? kXNone
+                           : C::LAYOUT == kLayHalf  ? (G > C::E ? kXShared : kXNone)
+                           : (G <= C::E / 2 ? kXNone : (G == C::D / 2 ? kXCrossHalf : kXAll));
+  static_assert(GL % 16 == 0, "group");
+};
+
+// Scale index within the vector of local group lg of thread t.
+template <class C, int G>
+__device__ __forceinline__ int global_group(int t, int lg) {
+  using Gr = Groups<C, G>;
+  if constexpr (Gr::X == kXNone) return global_y<C>(t, lg * Gr::GL) / G;
+  if constexpr (Gr::X == kXCrossHalf) return quarter_of(t, lg) / 2;
+  return 0;
+}
+
+// Whether thread t stores the scale of local group lg.
+template <class C, int G>
+__device__ __forceinline__ bool writes_scale(int t, int lg) {
+  using Gr = Groups<C, G>;
+  if constexpr (Gr::X == kXNone) return true;
+  if constexpr (Gr::X == kXAll) return t == 0 && lg == 0;
+  return t == 0;
+}
+
+template <class C, int G>
+__device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::NQ],
                                          float (&sc)[Groups<C, G>::NL]) {
   using Gr = Groups<C, G>;
+  constexpr int GP = Gr::GL / 2;  // pairs per local group
+  float m[Gr::NL];
+#pragma unroll
+  for (int g = 0; g < Gr::NL; ++g) m[g] = absmax2<GP>(&Y[g * GP]);
+  if constexpr (Gr::X == kXShared) {
+    m[0] = fmaxf(m[0], __shfl_xor_sync(kFull, m[0], 1));
+  } else if constexpr (Gr::X == kXCrossHalf) {
+    const float o0 = __shfl_xor_sync(kFull, m[0], 1), o1 = __shfl_xor_sync(kFull, m[1], 1);
+    m[0] = fmaxf(m[0], o1);
+    m[1] = fmaxf(m[1], o0);
+  } else if constexpr (Gr::X == kXAll) {
+    float a = fmaxf(m[0], m[1]);
+    a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
+    m[0] = a;
+    m[1] = a;
+  }
+  const f2 magic = mk2(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) {
-    float m = absmax<Gr::GL>(&Y[g * Gr::GL]);
-    if constexpr (Gr::SHARED) m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-    const float inv = m > 0.0f ? __fdiv_rn(7.0f, m) : 0.0f;
-    sc[g] = m * C::KAPPA7;
+    const float inv = m[g] > 0.0f ? __fdiv_rn(7.0f, m[g]) : 0.0f;
+    sc[g] = m[g] * C::KAPPA7;
+    const f2 inv2 = mk2(inv, inv);
 #pragma unroll
-    for (int w = 0; w < Gr::GL / 8; ++w) {
+    for (int w = 0; w < GP / 4; ++w) {
       uint32_t f[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        f[i] = __float_as_uint(__fmaf_rn(Y[g * Gr::GL + 8 * w + i], inv, kRoundMagic));
-      qw[(g * Gr::GL) / 8 + w] = pack8(f);
+      for (int i = 0; i < 4; ++i) {
+        const f2 r = fma2(Y[g * GP + 4 * w + i], inv2, magic);
+        f[2 * i] = __float_as_uint(lo2(r));
+        f[2 * i + 1] = __float_as_uint(hi2(r));
+      }
+      qw[(g * GP) / 4 + w] = pack8(f);
     }
   }
 }
@@ -399,17 +479,20 @@ __device__ __forceinline__ void quantize(const float (&Y)[C::E], uint32_t (&qw)[
 template <class C, int G>
 __device__ __forceinline__ void dequantize(const uint32_t (&qw)[C::NQ],
                                            const float (&sc)[Groups<C, G>::NL],
-                                           float (&Y)[C::E]) {
+                                           f2 (&Y)[C::P]) {
   using Gr = Groups<C, G>;
+  constexpr int GP = Gr::GL / 2;
+  const f2 magic = mk2(kUnpackMagic, kUnpackMagic);
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) {
     const float sk = sc[g] * C::KAPPA;
+    const f2 sk2 = mk2(sk, sk);
 #pragma unroll
-    for (int w = 0; w < Gr::GL / 8; ++w) {
-      float q[8];
-      unpack8(qw[(g * Gr::GL) / 8 + w], q);
+    for (int w = 0; w < GP / 4; ++w) {
+      f2 q[4];
+      unpack8(qw[(g * GP) / 4 + w], q);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) Y[g * Gr::GL + 8 * w + i] = q[i] * sk;
+      for (int i = 0; i < 4; ++i) Y[g * GP + 4 * w + i] = mul2(sub2(q[i], magic), sk2);
     }
   }
 }
@@ -452,19 +535,28 @@ template <class C, int G>
 __device__ __forceinline__ void store_scales_global(float* scales, int64_t vrow, int t,
                                                     const float (&sc)[Groups<C, G>::NL]) {
   using Gr = Groups<C, G>;
-  if constexpr (Gr::SHARED) {
-    if (t == 0) scales[vrow * Gr::NG] = sc[0];
-  } else {
-    float* p = scales + vrow * Gr::NG + t * Gr::NL;
-    if constexpr (Gr::NL == 1) {
-      p[0] = sc[0];
-    } else if constexpr (Gr::NL == 2) {
-      *reinterpret_cast<float2*>(p) = make_float2(sc[0], sc[1]);
-    } else {
+  float* row = scales + vrow * Gr::NG;
+  if constexpr (Gr::X == kXNone) {
+    // runs of R consecutive scales (two runs per thread in the quarter layout)
+    constexpr int R = C::LAYOUT == kLayQuarter ? Gr::NL / 2 : Gr::NL;
 #pragma unroll
-      for (int i = 0; i < Gr::NL; i += 4)
-        *reinterpret_cast<float4*>(p + i) = make_float4(sc[i], sc[i + 1], sc[i + 2], sc[i + 3]);
+    for (int r = 0; r < Gr::NL / R; ++r) {
+      float* p = row + global_group<C, G>(t, r * R);
+      if constexpr (R == 1) {
+        p[0] = sc[r];
+      } else if constexpr (R == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(sc[2 * r], sc[2 * r + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < R; i += 4)
+          *reinterpret_cast<float4*>(p + i) =
+              make_float4(sc[r * R + i], sc[r * R + i + 1], sc[r * R + i + 2], sc[r * R + i + 3]);
+      }
     }
+  } else {
+#pragma unroll
+    for (int lg = 0; lg < Gr::NL; ++lg)
+      if (writes_scale<C, G>(t, lg)) row[global_group<C, G>(t, lg)] = sc[lg];
   }
 }
 
@@ -472,9 +564,10 @@ template <class C, int G>
 __device__ __forceinline__ void load_scales_smem(uint32_t sbuf, int row, int t,
                                                  float (&sc)[Groups<C, G>::NL]) {
   using Gr = Groups<C, G>;
-  const uint32_t a = sbuf + uint32_t(row * Gr::NG + (Gr::SHARED ? 0 : t * Gr::NL)) * 4u;
+  const uint32_t a = sbuf + uint32_t(row * Gr::NG) * 4u;
 #pragma unroll
-  for (int i = 0; i < Gr::NL; ++i) sc[i] = __uint_as_float(lds32(a + 4 * i));
+  for (int lg = 0; lg < Gr::NL; ++lg)
+    sc[lg] = __uint_as_float(lds32(a + 4u * uint32_t(global_group<C, G>(t, lg))));
 }
 
 template <int S>
@@ -564,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue(nt);
       }
     }
-    float Y[C::E];
+    f2 Y[C::P];
     rotate_fwd<C>(xw, t, Y);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
@@ -662,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue(nt);
       }
     }
-    float Y[C::E];
+    f2 Y[C::P];
     dequantize<C, G>(qw, sc, Y);
     uint32_t xw[C::NW];
     rotate_inv<C>(Y, t, xw);
@@ -749,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     new_phase ^= 1u;
     uint32_t xw[C::NW];
     load_x<C>(xin, row, t, mask, xw);
-    float Y[C::E];
+    f2 Y[C::P];
     rotate_fwd<C>(xw, t, Y);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
@@ -758,12 +851,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t h = nt * C::VPW + row;
     if (h < a.n_heads) {
       float* p = a.scales + (h * a.cap + a.pos) * Gr::NG;
-      if constexpr (Gr::SHARED) {
-        if (t == 0) p[0] = sc[0];
-      } else {
 #pragma unroll
-        for (int i = 0; i < Gr::NL; ++i) p[t * Gr::NL + i] = sc[i];
-      }
+      for (int lg = 0; lg < Gr::NL; ++lg)
+        if (writes_scale<C, G>(t, lg)) p[global_group<C, G>(t, lg)] = sc[lg];
     }
     dequantize<C, G>(qw, sc, Y);
     rotate_inv<C>(Y, t, xw);
@@ -810,10 +900,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int head, tok;
       coords(i, head, tok);
       const int64_t r = int64_t(tok) + row;
-      const float* p = a.scales + (int64_t(head) * a.cap + r) * Gr::NG +
-                       (Gr::SHARED ? 0 : t * Gr::NL);
+      const float* p = a.scales + (int64_t(head) * a.cap + r) * Gr::NG;
 #pragma unroll
-      for (int k = 0; k < Gr::NL; ++k) sc[k] = r < a.pos ? __ldg(p + k) : 0.0f;
+      for (int k = 0; k < Gr::NL; ++k)
+        sc[k] = r < a.pos ? __ldg(p + global_group<C, G>(t, k)) : 0.0f;
     }
     const int s = int(ring.consumed % S_IN);
     const bool ok = mbar_wait_bounded(bars + 8u * s, uint32_t((ring.consumed / S_IN) & 1));
@@ -833,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue(ni);
       }
     }
-    float Y[C::E];
+    f2 Y[C::P];
     dequantize<C, G>(qw, sc, Y);
     uint32_t xw[C::NW];
     rotate_inv<C>(Y, t, xw);

@@ -271,38 +271,85 @@ __device__ __forceinline__ uint32_t float2_to_half2_bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// (dr + i di) * exp(-+ 2 pi i K / N), forward sign for INV = false.
+// A pair of floats in one 64-bit register pair, operated on by the sm_100
+// packed fp32 instructions (add/sub/mul/fma .rn.f32x2).  Complex numbers are
+// held as (re, im).
+struct f2 {
+  uint64_t v;
+};
+
+__device__ __forceinline__ f2 mk2(float x, float y) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ float lo2(f2 a) {
+  float x;
+  asm("mov.b64 {%0, _}, %1;" : "=f"(x) : "l"(a.v));
+  return x;
+}
+__device__ __forceinline__ float hi2(f2 a) {
+  float y;
+  asm("mov.b64 {_, %0}, %1;" : "=f"(y) : "l"(a.v));
+  return y;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+  f2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return r;
+}
+__device__ __forceinline__ f2 shfl_xor2(f2 a, int m) {
+  return mk2(__shfl_xor_sync(kFull, lo2(a), m), __shfl_xor_sync(kFull, hi2(a), m));
+}
+__device__ __forceinline__ f2 sel2(bool c, f2 a, f2 b) { return c ? a : b; }
+
+// max(a, b, c) in one instruction (three-operand max of sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// d * exp(-+ 2 pi i K / N), forward sign for INV = false.
 template <int N, int K, bool INV>
-__device__ __forceinline__ void twiddle(float dr, float di, float& outr, float& outi) {
+__device__ __forceinline__ f2 twiddle(f2 d) {
   if constexpr (K % N == 0) {
-    outr = dr;
-    outi = di;
+    return d;
   } else if constexpr (4 * K == N) {
-    if constexpr (!INV) {  // * (-i)
-      outr = di;
-      outi = -dr;
-    } else {  // * (+i)
-      outr = -di;
-      outi = dr;
-    }
+    const float x = lo2(d), y = hi2(d);
+    return INV ? mk2(-y, x) : mk2(y, -x);  // * (+i) : * (-i)
   } else {
     constexpr float c = tw_cos(K, N);
     constexpr float s = tw_sin(K, N);
+    const float x = lo2(d), y = hi2(d);
     if constexpr (!INV) {  // * (c - i s)
-      outr = fmaf(dr, c, di * s);
-      outi = fmaf(di, c, -(dr * s));
+      return mk2(fmaf(x, c, y * s), fmaf(y, c, -(x * s)));
     } else {  // * (c + i s)
-      outr = fmaf(dr, c, -(di * s));
-      outi = fmaf(di, c, dr * s);
+      return mk2(fmaf(x, c, -(y * s)), fmaf(y, c, x * s));
     }
   }
 }
 
-// In-place radix-2 DIF FFT of length N over (re, im) registers,
+// In-place radix-2 DIF FFT of length N over complex registers,
 // X_k = sum_n z_n exp(-+ 2 pi i k n / N) (no normalization).  Input in
 // natural order; X_k ends in slot bitrev(k).
 template <int N, bool INV>
-__device__ __forceinline__ void fft_dif(float (&re)[N], float (&im)[N]) {
+__device__ __forceinline__ void fft_dif(f2 (&z)[N]) {
   constexpr int L = ilog2(N);
   static_for<0, L>([&](auto st) {
     constexpr int h = N >> (decltype(st)::value + 1);
@@ -311,38 +358,47 @@ __device__ __forceinline__ void fft_dif(float (&re)[N], float (&im)[N]) {
       constexpr int o = bb % h;
       constexpr int i = (bb / h) * 2 * h + o;
       constexpr int j = i + h;
-      const float ar = re[i], ai = im[i], br = re[j], bi = im[j];
-      re[i] = ar + br;
-      im[i] = ai + bi;
-      twiddle<2 * h, o, INV>(ar - br, ai - bi, re[j], im[j]);
+      const f2 a = z[i], c = z[j];
+      z[i] = add2(a, c);
+      z[j] = twiddle<2 * h, o, INV>(sub2(a, c));
     });
   });
 }
 
-// In-place unnormalized Walsh-Hadamard transform (Sylvester order).
-template <int N>
-__device__ __forceinline__ void fwht(float (&v)[N]) {
-  static_for<0, ilog2(N)>([&](auto st) {
+// In-place unnormalized Walsh-Hadamard transform (Sylvester order) of the
+// 2P reals held as P pairs (element 2p in lo, 2p+1 in hi).
+template <int P>
+__device__ __forceinline__ void fwht(f2 (&v)[P]) {
+#pragma unroll
+  for (int p = 0; p < P; ++p) {  // h = 1: inside each pair
+    const float a = lo2(v[p]), b = hi2(v[p]);
+    v[p] = mk2(a + b, a - b);
+  }
+  static_for<0, ilog2(P)>([&](auto st) {  // h = 2, 4, ...: between pairs
     constexpr int h = 1 << decltype(st)::value;
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
+    for (int p = 0; p < P; ++p) {
+      if ((p & h) == 0) {
+        const f2 a = v[p], b = v[p + h];
+        v[p] = add2(a, b);
+        v[p + h] = sub2(a, b);
       }
     }
   });
 }
 
-// Max of |v[0..N)| as a balanced tree.
-template <int N>
-__device__ __forceinline__ float absmax(const float* v) {
-  if constexpr (N == 1) {
-    return fabsf(v[0]);
-  } else {
-    return fmaxf(absmax<N / 2>(v), absmax<N / 2>(v + N / 2));
+// Max of |x| over the 2P reals held in v[0..P).
+template <int P>
+__device__ __forceinline__ float absmax2(const f2* v) {
+  static_assert(P % 2 == 0, "pairs");
+  float m0 = fmaxf(fabsf(lo2(v[0])), fabsf(hi2(v[0])));
+  float m1 = fmaxf(fabsf(lo2(v[1])), fabsf(hi2(v[1])));
+#pragma unroll
+  for (int p = 2; p < P; p += 2) {
+    m0 = max3f(m0, fabsf(lo2(v[p])), fabsf(hi2(v[p])));
+    m1 = max3f(m1, fabsf(lo2(v[p + 1])), fabsf(hi2(v[p + 1])));
   }
+  return fmaxf(m0, m1);
 }
 
 // Eight round-to-int bit patterns (low byte = code) -> 8 packed nibbles:
@@ -355,15 +411,15 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&f)[8]) {
   return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
 }
 
-// Codes of a packed word as exact floats q in [-8, 7], element order.
-__device__ __forceinline__ void unpack8(uint32_t w, float (&q)[8]) {
+// Codes of a packed word, as 4 pairs of offset floats 2^23 + 8 + q
+// (element order: pair j = codes 2j, 2j+1).
+__device__ __forceinline__ void unpack8(uint32_t w, f2 (&q)[4]) {
   const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
   const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    q[2 * j] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + j)) - kUnpackMagic;
-    q[2 * j + 1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + j)) - kUnpackMagic;
-  }
+  for (int j = 0; j < 4; ++j)
+    q[j] = mk2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + j)),
+               __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + j)));
 }
 
 }  // namespace kvq

@@ -19,8 +19,8 @@ static __device__ unsigned g_status;
 template <int D>
 struct Tuning {
   static constexpr int TPV = DefaultTPV<D>::value;
-  static constexpr int FWD_STAGES = D == 64 ? 3 : 2;
-  static constexpr int INV_STAGES = 3;
+  static constexpr int FWD_STAGES = 2;
+  static constexpr int INV_STAGES = D == 64 ? 2 : 3;
 };
 
 namespace detail {
