@@ -279,6 +279,59 @@ def time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, warmup, samp
     return total, fwd, inv
 
 
+def run_e2e(kvq, x, signs, rot, g, packed, scales, out, world, steps, chunks=24):
+    n, d = x.shape
+    xh = x.cpu().pin_memory()
+    oh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    # chunk bounds on 32-row multiples keep every slice 16-byte aligned
+    bounds = [((i * n) // chunks) // 32 * 32 for i in range(chunks)] + [n]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(chunks)]
+    ev_run = [torch.cuda.Event() for _ in range(chunks)]
+    ev_out = [torch.cuda.Event() for _ in range(chunks)]
+
+    def one_pass():
+        for c in range(chunks):
+            a, b = bounds[c], bounds[c + 1]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_run[c])  # previous pass done reading x[a:b]
+                x[a:b].copy_(xh[a:b], non_blocking=True)
+                ev_in[c].record(s_in)
+            s_run.wait_event(ev_in[c])
+            s_run.wait_event(ev_out[c])  # previous pass done copying out[a:b]
+            kvq.kvq_rot_quant_fwd(x[a:b], signs, rot, g, packed[a:b], scales[a:b], s_run)
+            kvq.kvq_dequant_rot_inv(packed[a:b], scales[a:b], signs, rot, g, out[a:b], s_run)
+            ev_run[c].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_run[c])
+                oh[a:b].copy_(out[a:b], non_blocking=True)
+                ev_out[c].record(s_out)
+
+    e2e_steps = max(3, min(steps, 10))
+    for _ in range(2):
+        one_pass()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for st in (s_in, s_run, s_out):
+        st.wait_stream(cur)
+    for _ in range(e2e_steps):
+        one_pass()
+    for st in (s_in, s_run, s_out):
+        cur.wait_stream(st)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    if not torch.equal(oh[: bounds[1]], out[: bounds[1]].cpu()):
+        raise RuntimeError("end-to-end output differs from the device result")
+    e2e_ms = allreduce_max(e0.elapsed_time(e1), world)
+    fp16_bytes_step = 2 * n * d * 2
+    return {"value": world * e2e_steps * fp16_bytes_step / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 2),
+            "chunks": chunks, "gpu_launches_per_step": 2 * chunks}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -294,6 +347,8 @@ def main():
     ap.add_argument("--group", type=int, default=64)
     ap.add_argument("--n-vec", type=int, default=1 << 21)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--decode-pos", type=int, default=0,
+                    help="with --profile: run --reps 26-layer decode steps at this position")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.profile:
@@ -358,30 +413,10 @@ def main():
     detail["srht_inv_algo_gbs"] = algo / (i2 * 1e-3 / k2) / 1e9
     detail["srht_value_gbs"] = k2 * fp16_bytes_step / (t2 * 1e-3) / 1e9
 
-    # end to end through the public API with host buffers
-    e2e_steps = max(3, min(args.steps, 10))
-    xh = x.cpu().pin_memory()
-    oh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
-    stream = torch.cuda.current_stream()
-    for _ in range(2):
-        x.copy_(xh, non_blocking=True)
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
-        oh.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(xh, non_blocking=True)
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
-        oh.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = allreduce_max(e0.elapsed_time(e1), world)
-    e2e = {"value": world * e2e_steps * fp16_bytes_step / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
-           "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 2)}
+    # end to end through the public API with host buffers: the cache streams
+    # in chunks; host->device copy, forward+inverse and device->host copy of
+    # consecutive chunks run on three streams and overlap.
+    e2e = run_e2e(kvq, x, signs, rot, g, packed, scales, out, world, args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -423,6 +458,8 @@ def run_profile_case(args):
     recipe at (d, group, rot): the small case ncu captures."""
     from rotated_int4_kv_kvq_b200 import kvq
     dev = torch.device("cuda", 0)
+    if args.decode_pos > 0:
+        return run_profile_decode(kvq, dev, args)
     d, g = args.d, args.group
     tokens = 8192
     heads = max(1, -(-args.n_vec // (2 * tokens)))
@@ -439,6 +476,33 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": {"d": d, "group": g, "rot": args.rot,
                                        "n_vec": int(x.shape[0]), "reps": args.reps,
                                        "status": st}}))
+    if st != 0:
+        sys.exit(1)
+
+
+def run_profile_decode(kvq, dev, args):
+    """`reps` Gemma-3-1B-shaped decode steps (26 layers x K,V, d=256,
+    g=256, one call per layer) at position decode_pos."""
+    shape = W.scaled(W.config(4), tokens=args.decode_pos + 1)
+    d, g, L, pos = 256, 256, 26, args.decode_pos
+    seq = W.make_decode_sequence(shape, device=dev)
+    signs = torch.from_numpy(W.make_signs(d)).to(dev)
+    cap = pos + 1
+    packed = torch.zeros((2 * L, cap, d // 2), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((2 * L, cap, 1), dtype=torch.float32, device=dev)
+    p, s = kvq.kvq_rot_quant_fwd(seq.reshape(-1, d), signs, args.rot, g)
+    packed.copy_(p.reshape(2 * L, cap, -1))
+    scales.copy_(s.reshape(2 * L, cap, -1))
+    outs = [torch.empty((2, pos + 1, d), dtype=torch.float16, device=dev) for _ in range(L)]
+    xs = [seq[2 * l:2 * l + 2, pos].contiguous() for l in range(L)]
+    for _ in range(args.reps):
+        for l in range(L):
+            kvq.kvq_decode_step(xs[l], packed[2 * l:2 * l + 2], scales[2 * l:2 * l + 2], pos,
+                                signs, args.rot, g, outs[l])
+    torch.cuda.synchronize()
+    st = kvq.kvq_device_status()
+    print(json.dumps({"profile_decode": {"pos": pos, "rot": args.rot, "reps": args.reps,
+                                         "status": st}}))
     if st != 0:
         sys.exit(1)
 

@@ -26,6 +26,11 @@ SOURCES = ["kvq_api.cu", "kvq_d64.cu", "kvq_d128.cu", "kvq_d256.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+# Extra nvcc flags (e.g. -D tuning overrides) and an alternative output
+# path, for building variants side by side.
+EXTRA = os.environ.get("KVQ_NVCC_EXTRA", "").split()
+LIB = os.environ.get("KVQ_LIB_OUT", LIB)
+BUILD = os.environ.get("KVQ_BUILD_DIR", BUILD)
 
 
 def nvcc() -> str:
@@ -37,7 +42,7 @@ def nvcc() -> str:
 
 def _compile(src: str, ptxas_verbose: bool) -> tuple[str, str]:
     obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+    cmd = [nvcc(), *ARCH, *FLAGS, *EXTRA, "-c", os.path.join(CSRC, src), "-o", obj]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -54,7 +59,16 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+def _codelets() -> None:
+    """Regenerate kvq_rfft.cuh when the generator is newer than it."""
+    gen = os.path.join(CSRC, "gen_rfft.py")
+    out = os.path.join(CSRC, "kvq_rfft.cuh")
+    if not os.path.exists(out) or os.path.getmtime(gen) > os.path.getmtime(out):
+        subprocess.run([sys.executable, gen], check=True, capture_output=True)
+
+
 def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
+    _codelets()
     if not force and not _stale():
         return LIB
     os.makedirs(BUILD, exist_ok=True)

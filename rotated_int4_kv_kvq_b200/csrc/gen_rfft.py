@@ -1,0 +1,418 @@
+"""Generate straight-line real-input FFT codelets for libkvq (kvq_rfft.cuh).
+
+    python rotated_int4_kv_kvq_b200/csrc/gen_rfft.py
+
+For n in {64, 128} it emits
+
+  rfft<n>(x, y):  y[0] = X_0/sqrt2, y[1] = X_{n/2}/sqrt2,
+                  y[2k] = Re X_k, y[2k+1] = Im X_k   (1 <= k < n/2),
+                  X_k = sum_m x_m exp(-2 pi i k m / n)  (unnormalized);
+  irfft<n>(y, x): the transpose map, x_m = sum_k X_k exp(+2 pi i k m / n)
+                  with X rebuilt from y in the same packing (X_0 = sqrt2 y[0],
+                  X_{n/2} = sqrt2 y[1]).
+
+The transforms follow the split-radix decomposition for real data (even
+samples through a half-length real DFT, samples 4m+1 and 4m+3 through two
+quarter-length real DFTs, recombined with twiddles W^k and W^3k), keeping
+only the non-redundant half of every Hermitian spectrum.  The generator
+builds an expression graph with hash-consing, folds trivial twiddles
+(+-1, +-i) and negations into add/sub, writes twiddle products as fused
+multiply-adds, and checks the graph numerically against numpy's FFT before
+emitting anything.  Twiddle constants are cos/sin evaluated in double and
+rounded once to float.
+"""
+
+from __future__ import annotations
+
+import math
+import os
+import sys
+
+import numpy as np
+
+
+class R:
+    """A real value: `sign * node`, node None meaning exactly zero."""
+
+    __slots__ = ("node", "sign")
+
+    def __init__(self, node, sign=1):
+        self.node = node
+        self.sign = sign
+
+
+ZERO = R(None, 1)
+
+
+class Graph:
+    def __init__(self):
+        self.nodes = []  # (op, args)
+        self.memo = {}
+
+    def _mk(self, op, *args):
+        key = (op, args)
+        if key not in self.memo:
+            self.memo[key] = len(self.nodes)
+            self.nodes.append(key)
+        return self.memo[key]
+
+    def inp(self, name):
+        return R(self._mk("in", name))
+
+    @staticmethod
+    def neg(a):
+        return R(a.node, -a.sign)
+
+    def add(self, a, b):
+        if a.node is None:
+            return b
+        if b.node is None:
+            return a
+        if a.sign == b.sign:
+            lo, hi = sorted((a.node, b.node))
+            return R(self._mk("add", lo, hi), a.sign)
+        if a.node == b.node:
+            return ZERO
+        pos, neg_ = (a, b) if a.sign > 0 else (b, a)
+        return R(self._mk("sub", pos.node, neg_.node), 1)
+
+    def sub(self, a, b):
+        return self.add(a, self.neg(b))
+
+    def mulc(self, a, c):
+        if a.node is None or c == 0.0:
+            return ZERO
+        if c == 1.0:
+            return a
+        if c == -1.0:
+            return self.neg(a)
+        s = a.sign * (1 if c > 0 else -1)
+        return R(self._mk("mul", a.node, abs(c)), s)
+
+    def fmac(self, a, c, b):
+        """a * c + b with c a constant (one fused multiply-add)."""
+        if a.node is None or c == 0.0:
+            return b
+        if b.node is None:
+            return self.mulc(a, c)
+        if c in (1.0, -1.0):
+            return self.add(self.mulc(a, c), b)
+        cc = a.sign * b.sign * c
+        return R(self._mk("fma", a.node, cc, b.node), b.sign)
+
+    # complex helpers: values are (re, im) pairs of R
+    def cadd(self, a, b):
+        return (self.add(a[0], b[0]), self.add(a[1], b[1]))
+
+    def csub(self, a, b):
+        return (self.sub(a[0], b[0]), self.sub(a[1], b[1]))
+
+    @staticmethod
+    def conj(a):
+        return (a[0], Graph.neg(a[1]))
+
+    @staticmethod
+    def mul_i(a):  # i * a
+        return (Graph.neg(a[1]), a[0])
+
+    @staticmethod
+    def mul_mi(a):  # -i * a
+        return (a[1], Graph.neg(a[0]))
+
+    def ctw(self, a, k, n, sign):
+        """a * exp(sign * 2 pi i k / n), folding the trivial angles."""
+        k %= n
+        if k == 0:
+            return a
+        if 4 * k == n:
+            return self.mul_i(a) if sign > 0 else self.mul_mi(a)
+        if 2 * k == n:
+            return (self.neg(a[0]), self.neg(a[1]))
+        if 4 * k == 3 * n:
+            return self.mul_mi(a) if sign > 0 else self.mul_i(a)
+        ang = 2.0 * math.pi * k / n
+        c = float(np.float32(math.cos(ang)))
+        s = float(np.float32(sign * math.sin(ang)))
+        # (ar + i ai)(c + i s) = (ar c - ai s) + i (ar s + ai c)
+        re = self.fmac(a[0], c, self.mulc(a[1], -s))
+        im = self.fmac(a[0], s, self.mulc(a[1], c))
+        return (re, im)
+
+
+def rdft(g: Graph, x):
+    """Real DFT of x (list of R, len n): returns X_k as (re, im) for
+    k = 0..n/2 (X_0 and X_{n/2} real)."""
+    n = len(x)
+    if n == 1:
+        return [(x[0], ZERO)]
+    if n == 2:
+        return [(g.add(x[0], x[1]), ZERO), (g.sub(x[0], x[1]), ZERO)]
+    e = rdft(g, x[0::2])  # n/2: k = 0..n/4
+    u = rdft(g, x[1::4])  # n/4: k = 0..n/8
+    v = rdft(g, x[3::4])
+
+    def full(h, m, k):  # value at k of a Hermitian spectrum of length m
+        k %= m
+        return h[k] if k <= m // 2 else Graph.conj(h[m - k])
+
+    out = [None] * (n // 2 + 1)
+    q = n // 4
+    # A_k = W^k U_k, B_k = W^3k V_k for k <= n/8; the rest by symmetry:
+    # A_{q-k} = -i conj(A_k), B_{q-k} = +i conj(B_k).
+    a = {}
+    b = {}
+    for k in range(0, n // 8 + 1):
+        a[k] = g.ctw(full(u, q, k), k, n, -1)
+        b[k] = g.ctw(full(v, q, k), 3 * k, n, -1)
+    for k in range(n // 8 + 1, q):
+        a[k] = Graph.mul_mi(Graph.conj(a[q - k]))
+        b[k] = Graph.mul_i(Graph.conj(b[q - k]))
+    for k in range(0, q):
+        s = g.cadd(a[k], b[k])
+        dd = g.csub(a[k], b[k])
+        out[k] = g.cadd(full(e, n // 2, k), s)
+        out[k + q] = g.cadd(full(e, n // 2, k + q), Graph.mul_mi(dd))
+    s0 = g.cadd(a[0], b[0])
+    out[n // 2] = g.csub(full(e, n // 2, 0), s0)
+    return out
+
+
+def irdft(g: Graph, xs):
+    """Inverse of rdft's spectrum: xs = X_k for k = 0..n/2 (Hermitian);
+    returns x_m = sum_{k<n} X_k exp(+2 pi i k m / n), m = 0..n-1."""
+    n = 2 * (len(xs) - 1)
+    if n == 1 or len(xs) == 1:
+        return [xs[0][0]]
+    if n == 2:
+        return [g.add(xs[0][0], xs[1][0]), g.sub(xs[0][0], xs[1][0])]
+
+    def full(k):
+        k %= n
+        return xs[k] if k <= n // 2 else Graph.conj(xs[n - k])
+
+    q = n // 4
+    ep = [g.cadd(full(k), full(k + n // 2)) for k in range(0, q + 1)]
+    up, vp = [], []
+    for k in range(0, n // 8 + 1):
+        d1 = g.csub(full(k), full(k + n // 2))
+        d2 = g.csub(full(k + q), full(k + 3 * q))
+        up.append(g.ctw(g.cadd(d1, Graph.mul_i(d2)), k, n, +1))
+        vp.append(g.ctw(g.csub(d1, Graph.mul_i(d2)), 3 * k, n, +1))
+    xe = irdft(g, ep)
+    xu = irdft(g, up)
+    xv = irdft(g, vp)
+    x = [None] * n
+    x[0::2] = xe
+    x[1::4] = xu
+    x[3::4] = xv
+    return x
+
+
+R2 = float(np.float32(math.sqrt(2.0)))
+R2I = float(np.float32(1.0 / math.sqrt(2.0)))
+
+
+def build_forward(n):
+    g = Graph()
+    x = [g.inp(f"x[{i}]") for i in range(n)]
+    xs = rdft(g, x)
+    outs = [g.mulc(xs[0][0], R2I), g.mulc(xs[n // 2][0], R2I)]
+    for k in range(1, n // 2):
+        outs += [xs[k][0], xs[k][1]]
+    return g, outs
+
+
+def build_inverse(n):
+    g = Graph()
+    y = [g.inp(f"y[{i}]") for i in range(n)]
+    xs = [(g.mulc(y[0], R2), ZERO)]
+    xs += [(y[2 * k], y[2 * k + 1]) for k in range(1, n // 2)]
+    xs += [(g.mulc(y[1], R2), ZERO)]
+    outs = irdft(g, xs)
+    return g, outs
+
+
+def evaluate(g: Graph, outs, inputs: dict):
+    vals = {}
+    for i, (op, args) in enumerate(g.nodes):
+        if op == "in":
+            vals[i] = inputs[args[0]]
+        elif op == "add":
+            vals[i] = vals[args[0]] + vals[args[1]]
+        elif op == "sub":
+            vals[i] = vals[args[0]] - vals[args[1]]
+        elif op == "mul":
+            vals[i] = vals[args[0]] * args[1]
+        elif op == "fma":
+            vals[i] = vals[args[0]] * args[1] + vals[args[2]]
+    res = []
+    for o in outs:
+        res.append(0.0 if o.node is None else o.sign * vals[o.node])
+    return np.array(res)
+
+
+def live_nodes(g: Graph, outs):
+    live = set()
+    stack = [o.node for o in outs if o.node is not None]
+    while stack:
+        i = stack.pop()
+        if i in live:
+            continue
+        live.add(i)
+        op, args = g.nodes[i]
+        if op in ("add", "sub"):
+            stack += [args[0], args[1]]
+        elif op == "mul":
+            stack.append(args[0])
+        elif op == "fma":
+            stack += [args[0], args[2]]
+    return live
+
+
+def check(n):
+    rng = np.random.default_rng(n)
+    xv = rng.standard_normal((4, n))
+    g, outs = build_forward(n)
+    X = np.fft.rfft(xv, axis=1)
+    for r in range(4):
+        got = evaluate(g, outs, {f"x[{i}]": xv[r, i] for i in range(n)})
+        ref = np.empty(n)
+        ref[0] = X[r, 0].real / math.sqrt(2)
+        ref[1] = X[r, n // 2].real / math.sqrt(2)
+        ref[2::2] = X[r, 1:n // 2].real
+        ref[3::2] = X[r, 1:n // 2].imag
+        err = np.abs(got - ref).max() / np.abs(ref).max()
+        assert err < 1e-6, (n, "forward", err)
+    gi, outi = build_inverse(n)
+    for r in range(4):
+        yv = rng.standard_normal(n)
+        got = evaluate(gi, outi, {f"y[{i}]": yv[i] for i in range(n)})
+        Xs = np.zeros(n // 2 + 1, complex)
+        Xs[0] = yv[0] * math.sqrt(2)
+        Xs[n // 2] = yv[1] * math.sqrt(2)
+        Xs[1:n // 2] = yv[2::2][: n // 2 - 1] + 1j * yv[3::2][: n // 2 - 1]
+        ref = np.fft.irfft(Xs, n) * n
+        err = np.abs(got - ref).max() / np.abs(ref).max()
+        assert err < 1e-6, (n, "inverse", err)
+
+
+def fmt(c: float) -> str:
+    return f"{np.float32(c).item():.9e}f"
+
+
+def use_counts(g: Graph, outs, live):
+    uses = {i: 0 for i in live}
+    for i in live:
+        op, args = g.nodes[i]
+        if op in ("add", "sub"):
+            uses[args[0]] += 1
+            uses[args[1]] += 1
+        elif op == "mul":
+            uses[args[0]] += 1
+        elif op == "fma":
+            uses[args[0]] += 1
+            uses[args[2]] += 1
+    for o in outs:
+        if o.node is not None:
+            uses[o.node] += 1
+    return uses
+
+
+def emit(name, g: Graph, outs, in_arr, out_arr, n):
+    """Straight-line code; an add/sub whose operand is a product used only
+    there is emitted as one fused multiply-add."""
+    live = live_nodes(g, outs)
+    uses = use_counts(g, outs, live)
+    fused = {}  # add/sub node -> (mul operand index, other operand, sign of other)
+    absorbed = set()
+    for i in sorted(live):
+        op, args = g.nodes[i]
+        if op not in ("add", "sub"):
+            continue
+        for pos in (1, 0) if op == "add" else (1, 0):
+            m = args[pos]
+            mop, margs = g.nodes[m]
+            if mop == "mul" and uses[m] == 1 and m not in absorbed:
+                other = args[1 - pos]
+                # add: m + other; sub: args[0] - args[1]
+                if op == "add":
+                    fused[i] = (m, +1, other, +1)
+                elif pos == 1:  # other - m
+                    fused[i] = (m, -1, other, +1)
+                else:  # m - other
+                    fused[i] = (m, +1, other, -1)
+                absorbed.add(m)
+                break
+    lines = [f"__device__ __forceinline__ void {name}(const float (&{in_arr})[{n}], "
+             f"float (&{out_arr})[{n}]) {{"]
+    counts = {"add": 0, "sub": 0, "mul": 0, "fma": 0}
+
+    def ref(i):
+        op, args = g.nodes[i]
+        return args[0] if op == "in" else f"t{i}"
+
+    for i, (op, args) in enumerate(g.nodes):
+        if i not in live or op == "in" or i in absorbed:
+            continue
+        if i in fused:
+            m, msign, other, osign = fused[i]
+            src, c = g.nodes[m][1]
+            e = f"fmaf({ref(src)}, {fmt(msign * c)}, {'-' if osign < 0 else ''}{ref(other)})"
+            counts["fma"] += 1
+        elif op == "add":
+            e = f"{ref(args[0])} + {ref(args[1])}"
+            counts["add"] += 1
+        elif op == "sub":
+            e = f"{ref(args[0])} - {ref(args[1])}"
+            counts["sub"] += 1
+        elif op == "mul":
+            e = f"{ref(args[0])} * {fmt(args[1])}"
+            counts["mul"] += 1
+        else:
+            e = f"fmaf({ref(args[0])}, {fmt(args[1])}, {ref(args[2])})"
+            counts["fma"] += 1
+        lines.append(f"  const float t{i} = {e};")
+    for j, o in enumerate(outs):
+        if o.node is None:
+            lines.append(f"  {out_arr}[{j}] = 0.0f;")
+        else:
+            lines.append(f"  {out_arr}[{j}] = {'-' if o.sign < 0 else ''}{ref(o.node)};")
+    lines.append("}")
+    total = sum(counts.values())
+    head = (f"// {name}: {counts['add'] + counts['sub']} add/sub, {counts['mul']} mul, "
+            f"{counts['fma']} fma ({total} fp32 instructions)")
+    return head + "\n" + "\n".join(lines) + "\n", total
+
+
+def main(path=None):
+    here = os.path.dirname(os.path.abspath(__file__))
+    path = path or os.path.join(here, "kvq_rfft.cuh")
+    parts = [
+        "// kvq_rfft.cuh -- GENERATED by gen_rfft.py; do not edit by hand.\n",
+        "// Real-input split-radix FFT codelets (see gen_rfft.py for the maps).\n",
+        "#pragma once\n\nnamespace kvq {\n\n",
+        "template <int N> struct RFFT;\n\n",
+    ]
+    for n in (64, 128):
+        check(n)
+        gf, of = build_forward(n)
+        gi, oi = build_inverse(n)
+        fwd, cf = emit(f"rfft{n}_fwd", gf, of, "x", "y", n)
+        inv, ci = emit(f"rfft{n}_inv", gi, oi, "y", "x", n)
+        parts += [fwd, "\n", inv, "\n"]
+        parts.append(
+            f"template <> struct RFFT<{n}> {{\n"
+            f"  static __device__ __forceinline__ void fwd(const float (&x)[{n}], float (&y)[{n}]) "
+            f"{{ rfft{n}_fwd(x, y); }}\n"
+            f"  static __device__ __forceinline__ void inv(const float (&y)[{n}], float (&x)[{n}]) "
+            f"{{ rfft{n}_inv(y, x); }}\n"
+            f"}};\n\n")
+        print(f"n={n}: forward {cf} fp32 ops, inverse {ci} fp32 ops", file=sys.stderr)
+    parts.append("}  // namespace kvq\n")
+    with open(path, "w") as f:
+        f.write("".join(parts))
+    return path
+
+
+if __name__ == "__main__":
+    main()

@@ -21,6 +21,13 @@
 #pragma once
 
 #include "kvq_device.cuh"
+#include "kvq_rfft.cuh"
+
+// Inverse of the one-thread SRFT: 1 = generated c2r codelet, 0 = half-length
+// complex FFT with the real pre-split.
+#ifndef KVQ_INV_CODELET
+#define KVQ_INV_CODELET 0
+#endif
 
 namespace kvq {
 
@@ -52,11 +59,20 @@ struct Cfg {
   static constexpr int SLAB = VPW * 128;   // one 64-column fp16 slab
   static constexpr int QP = D / 2;         // code row pitch in bytes
   static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
-  // y = KAPPA * (unnormalized transform of u): SRFT 1/sqrt(2d), SRHT 1/sqrt(d)
-  static constexpr double KAPPA_D =
-      ROT == kRotSRFT ? 1.0 / const_sqrt(2.0 * D) : 1.0 / const_sqrt(double(D));
-  static constexpr float KAPPA = float(KAPPA_D);
-  static constexpr float KAPPA7 = float(KAPPA_D / 7.0);
+  // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
+  // takes Yin = KAPPA_INV * y_hat.  One-thread SRFT (generated real-FFT
+  // codelets, Y = packed rfft with X_0, X_{d/2} over sqrt2): sqrt(2/d) and
+  // 1/sqrt(2d).  Thread-pair SRFT (Y = 2X packing): 1/sqrt(2d) both ways.
+  // SRHT: 1/sqrt(d) both ways.
+  static constexpr bool CODELET = ROT == kRotSRFT && TPV == 1;
+  static constexpr bool INV_CODELET = KVQ_INV_CODELET != 0;
+  static constexpr double KAPPA_FWD_D =
+      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D))
+                      : (CODELET ? const_sqrt(2.0 / D) : 1.0 / const_sqrt(2.0 * D));
+  static constexpr double KAPPA_INV_D =
+      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : 1.0 / const_sqrt(2.0 * D);
+  static constexpr float KAPPA_INV = float(KAPPA_INV_D);
+  static constexpr float KAPPA7 = float(KAPPA_FWD_D / 7.0);
   static_assert(D % 64 == 0 && (TPV == 1 || TPV == 2), "shape");
 };
 
@@ -212,37 +228,17 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
       for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
     }
   } else if constexpr (C::TPV == 1) {
-    // z_n = u_{2n} + i u_{2n+1}; Z = FFT_{d/2}(z); X_k from (Z_k, Z_{d/2-k}).
-    constexpr int N = C::D / 2;
-    constexpr int LN = ilog2(N);
-    f2 z[N];
+    // Real-input split-radix codelet: Y = packed rfft of u.
+    float u[C::D], y[C::D];
 #pragma unroll
-    for (int j = 0; j < N; ++j) {
+    for (int j = 0; j < C::NW; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
-      z[j] = mk2(f.x, f.y);
+      u[2 * j] = f.x;
+      u[2 * j + 1] = f.y;
     }
-    fft_dif<N, false>(z);
-    {
-      const float a = lo2(z[0]), b = hi2(z[0]);
-      Y[0] = mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));  // sqrt2 X_0, sqrt2 X_{d/2}
-    }
-    static_for<1, N / 2>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      // P1 = Z_k + Z_{N-k} = (Sr, Ti), P2 = Z_k - Z_{N-k} = (Tr, Si) where
-      // S = Z_k + conj Z_{N-k} = 2E_k and T = Z_k - conj Z_{N-k} = 2i O_k.
-      const f2 p1 = add2(z[bitrev(k, LN)], z[bitrev(N - k, LN)]);
-      const f2 p2 = sub2(z[bitrev(k, LN)], z[bitrev(N - k, LN)]);
-      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
-      // W^k (-i T), W = exp(-2 pi i / d)
-      constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float wr = fmaf(c, ti, -(s * tr)), wi = -fmaf(c, tr, s * ti);
-      Y[k] = mk2(sr + wr, si + wi);          // 2 X_k
-      Y[N - k] = mk2(sr - wr, wi - si);      // 2 X_{N-k} = conj(S - W^k (-i T))
-    });
-    {
-      const f2 zm = z[bitrev(N / 2, LN)];
-      Y[N / 2] = mk2(2.0f * lo2(zm), -2.0f * hi2(zm));  // 2 X_{d/4} = 2 conj Z_{d/4}
-    }
+    RFFT<C::D>::fwd(u, y);
+#pragma unroll
+    for (int k = 0; k < C::P; ++k) Y[k] = mk2(y[2 * k], y[2 * k + 1]);
   } else {
     // Thread pair, d/2 = N complex points, M = N/2 per thread, Q = M/2.
     // Thread t holds z_{2m+t}: in-thread FFT_M gives F_t(k); thread 1 turns
@@ -322,7 +318,18 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     fwht<C::P>(Y);
 #pragma unroll
     for (int j = 0; j < C::NW; ++j) xw[j] = float2_to_half2_bits(lo2(Y[j]), hi2(Y[j]));
+  } else if constexpr (C::TPV == 1 && C::INV_CODELET) {
+    float y[C::D], u[C::D];
+#pragma unroll
+    for (int k = 0; k < C::P; ++k) {
+      y[2 * k] = lo2(Y[k]);
+      y[2 * k + 1] = hi2(Y[k]);
+    }
+    RFFT<C::D>::inv(y, u);
+#pragma unroll
+    for (int n = 0; n < C::NW; ++n) xw[n] = float2_to_half2_bits(u[2 * n], u[2 * n + 1]);
   } else if constexpr (C::TPV == 1) {
+    // Half-length complex inverse FFT after the real pre-split.
     constexpr int N = C::D / 2;
     constexpr int LN = ilog2(N);
     f2 z[N];
@@ -466,9 +473,15 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
       uint32_t f[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const f2 r = fma2(Y[g * GP + 4 * w + i], inv2, magic);
-        f[2 * i] = __float_as_uint(lo2(r));
-        f[2 * i + 1] = __float_as_uint(hi2(r));
+        const f2 v = Y[g * GP + 4 * w + i];
+        if constexpr (C::CODELET) {  // scalar outputs: no re-pairing moves
+          f[2 * i] = __float_as_uint(__fmaf_rn(lo2(v), inv, kRoundMagic));
+          f[2 * i + 1] = __float_as_uint(__fmaf_rn(hi2(v), inv, kRoundMagic));
+        } else {
+          const f2 r = fma2(v, inv2, magic);
+          f[2 * i] = __float_as_uint(lo2(r));
+          f[2 * i + 1] = __float_as_uint(hi2(r));
+        }
       }
       qw[(g * GP) / 4 + w] = pack8(f);
     }
@@ -485,7 +498,7 @@ __device__ __forceinline__ void dequantize(const uint32_t (&qw)[C::NQ],
   const f2 magic = mk2(kUnpackMagic, kUnpackMagic);
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) {
-    const float sk = sc[g] * C::KAPPA;
+    const float sk = sc[g] * C::KAPPA_INV;
     const f2 sk2 = mk2(sk, sk);
 #pragma unroll
     for (int w = 0; w < GP / 4; ++w) {
@@ -590,8 +603,8 @@ __device__ __noinline__ void drain_and_fail(uint32_t bars, const Ring& r, unsign
   atomicOr(status, 1u);
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, int ROT, int TPV, int S_IN, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     kvq_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                    const FwdArgs a, unsigned* status) {
   using C = Cfg<D, ROT, TPV>;
@@ -683,8 +696,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, int ROT, int TPV, int S_IN, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     kvq_inv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmX, const InvArgs a, unsigned* status) {
   using C = Cfg<D, ROT, TPV>;
@@ -784,8 +797,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (forward step), write its codes/scales into cache row `pos`, and write
 // its dequantized output row from registers; the remaining tiles run the
 // inverse step over cache rows [0, pos) of one head each.
-template <int D, int G, int ROT, int TPV, int S_IN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, int ROT, int TPV, int S_IN, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     kvq_decode_kernel(const __grid_constant__ CUtensorMap tmXn,  // x_new [n_heads][d]
                       const __grid_constant__ CUtensorMap tmQn,  // packed row pos, per head
                       const __grid_constant__ CUtensorMap tmOn,  // out row pos, per head

@@ -16,11 +16,39 @@ namespace kvq {
 // Bit 0: a bounded wait on an asynchronous copy ran out.
 static __device__ unsigned g_status;
 
+// Per-d launch tuning: pipeline depth (tiles in flight per warp) and the
+// minimum resident blocks per SM the register allocation must allow.
+#ifndef KVQ_FWD_MINB_64
+#define KVQ_FWD_MINB_64 4
+#endif
+#ifndef KVQ_INV_MINB_64
+#define KVQ_INV_MINB_64 4
+#endif
+#ifndef KVQ_FWD_MINB_128
+#define KVQ_FWD_MINB_128 2
+#endif
+#ifndef KVQ_INV_MINB_128
+#define KVQ_INV_MINB_128 2
+#endif
+#ifndef KVQ_FWD_MINB_256
+#define KVQ_FWD_MINB_256 2
+#endif
+#ifndef KVQ_INV_MINB_256
+#define KVQ_INV_MINB_256 2
+#endif
+#ifndef KVQ_INV_STAGES_64
+#define KVQ_INV_STAGES_64 2
+#endif
+
 template <int D>
 struct Tuning {
   static constexpr int TPV = DefaultTPV<D>::value;
   static constexpr int FWD_STAGES = 2;
-  static constexpr int INV_STAGES = D == 64 ? 2 : 3;
+  static constexpr int INV_STAGES = D == 64 ? KVQ_INV_STAGES_64 : 3;
+  static constexpr int FWD_MINB =
+      D == 64 ? KVQ_FWD_MINB_64 : (D == 128 ? KVQ_FWD_MINB_128 : KVQ_FWD_MINB_256);
+  static constexpr int INV_MINB =
+      D == 64 ? KVQ_INV_MINB_64 : (D == 128 ? KVQ_INV_MINB_128 : KVQ_INV_MINB_256);
 };
 
 namespace detail {
@@ -81,7 +109,7 @@ inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
 template <int D, int G, int ROT>
 cudaError_t fwd_one(const FwdLaunch& L) {
   using T = Tuning<D>;
-  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES>;
+  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::FWD_MINB>;
   constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES>();
   int occ;
   unsigned* st;
@@ -97,7 +125,7 @@ cudaError_t fwd_one(const FwdLaunch& L) {
 template <int D, int G, int ROT>
 cudaError_t inv_one(const InvLaunch& L) {
   using T = Tuning<D>;
-  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES>;
+  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::INV_MINB>;
   constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES>();
   int occ;
   unsigned* st;
@@ -114,7 +142,7 @@ cudaError_t inv_one(const InvLaunch& L) {
 template <int D, int G, int ROT>
 cudaError_t decode_one(const DecodeLaunch& L) {
   using T = Tuning<D>;
-  constexpr auto kern = kvq_decode_kernel<D, G, ROT, T::TPV, T::INV_STAGES>;
+  constexpr auto kern = kvq_decode_kernel<D, G, ROT, T::TPV, T::INV_STAGES, 1>;
   constexpr int smem = decode_smem_bytes<D, ROT, T::TPV, T::INV_STAGES>();
   int occ;
   unsigned* st;

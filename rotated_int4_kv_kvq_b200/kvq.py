@@ -24,7 +24,8 @@ STATUS = {
     7: "KVQ_ERR_BAD_SIZE", 8: "KVQ_ERR_DEVICE_TIMEOUT", 9: "KVQ_ERR_UNSUPPORTED_DEVICE",
 }
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
+LIB_PATH = os.environ.get("KVQ_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
 EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_decode_step",
            "kvq_status_string", "kvq_device_status", "kvq_version")
