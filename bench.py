@@ -357,6 +357,9 @@ def main():
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
 
     from rotated_int4_kv_kvq_b200 import kvq

@@ -186,6 +186,14 @@ kvq_status kvq_decode_step(const uint16_t* x_new, uint8_t* packed, float* scales
   if (n_heads == 0) return KVQ_OK;
   DeviceInfo dev;
   if (kvq_status s = device_info(&dev)) return s;
+  if (n_heads * (pos + 1) <= kvq::kWideMaxRows) {  // latency path: a warp per vector
+    kvq::DecodeWideLaunch W{x_new, packed, scales, out, signs, n_heads, cap, pos, dev.sm_count,
+                            reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = d == 64    ? kvq::launch_decode_wide<64>(group, rot, W)
+                    : d == 128 ? kvq::launch_decode_wide<128>(group, rot, W)
+                               : kvq::launch_decode_wide<256>(group, rot, W);
+    return from_cuda(e);
+  }
   const uint64_t qp = uint64_t(d / 2), xp = uint64_t(2 * d);
   const uint64_t H = uint64_t(n_heads), CAP = uint64_t(cap), P = uint64_t(pos);
   CUtensorMap tmXn, tmQn, tmOn, tmQc, tmOc;

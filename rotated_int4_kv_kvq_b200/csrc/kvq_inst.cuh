@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "kvq_codec.cuh"
+#include "kvq_wide.cuh"
 #include "kvq_launch.h"
 
 namespace kvq {
@@ -164,6 +165,35 @@ cudaError_t decode_one(const DecodeLaunch& L) {
   return cudaGetLastError();
 }
 
+template <int D, int G, int ROT>
+cudaError_t decode_wide_one(const DecodeWideLaunch& L) {
+  constexpr auto kern = kvq_decode_wide_kernel<D, G, ROT>;
+  constexpr int threads = 256;
+  int occ;
+  cudaError_t e;
+  {
+    static int occ_dev[kMaxDevices];
+    static std::mutex mu;
+    int dev;
+    e = current_device(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    if (occ_dev[dev] == 0) {
+      int b = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, threads, 0);
+      if (e != cudaSuccess) return e;
+      occ_dev[dev] = std::max(b, 1);
+    }
+    occ = occ_dev[dev];
+  }
+  DecodeWideArgs a{L.x_new, L.packed, L.scales, L.out, L.signs, L.n_heads, L.cap, L.pos};
+  const int64_t rows = L.n_heads * (L.pos + 1);
+  const int64_t want = (rows + threads / 32 - 1) / (threads / 32);
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(L.sm_count) * occ)));
+  kern<<<grid, threads, 0, L.stream>>>(a);
+  return cudaGetLastError();
+}
+
 // Run Op<D, G, ROT>(launch) for the runtime (group, rot) pair.
 template <int D, template <int, int, int> class Op, class L>
 cudaError_t dispatch(int group, int rot, const L& l) {
@@ -196,6 +226,10 @@ template <int D, int G, int ROT>
 struct DecodeOp {
   static cudaError_t run(const DecodeLaunch& l) { return decode_one<D, G, ROT>(l); }
 };
+template <int D, int G, int ROT>
+struct DecodeWideOp {
+  static cudaError_t run(const DecodeWideLaunch& l) { return decode_wide_one<D, G, ROT>(l); }
+};
 
 }  // namespace detail
 
@@ -212,6 +246,11 @@ cudaError_t launch_inv(int group, int rot, const InvLaunch& L) {
 template <int D>
 cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L) {
   return detail::dispatch<D, detail::DecodeOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L) {
+  return detail::dispatch<D, detail::DecodeWideOp>(group, rot, L);
 }
 
 template <int D>

@@ -34,6 +34,21 @@ struct InvLaunch {
   cudaStream_t stream;
 };
 
+// Decode calls with at most this many rows (new tokens + cached rows) run
+// the one-warp-per-vector kernel (latency); larger ones the tiled kernel.
+constexpr int64_t kWideMaxRows = int64_t(1) << 16;
+
+struct DecodeWideLaunch {
+  const uint16_t* x_new;
+  uint8_t* packed;
+  float* scales;
+  uint16_t* out;
+  const int8_t* signs;
+  int64_t n_heads, cap, pos;
+  int sm_count;
+  cudaStream_t stream;
+};
+
 struct DecodeLaunch {
   const CUtensorMap* tmXn;  // x_new [n_heads][d], box {64, VPW}
   const CUtensorMap* tmQn;  // packed row pos of every head, box {d/2, VPW}
@@ -54,6 +69,8 @@ template <int D>
 cudaError_t launch_inv(int group, int rot, const InvLaunch& L);
 template <int D>
 cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L);
+template <int D>
+cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L);
 // Reads (and optionally clears) the device status word of that translation
 // unit on the current device; the caller has synchronized the device.
 template <int D>

@@ -38,16 +38,13 @@ def make_cache(kvq, heads, cap, pos, d, group, rot, signs, seed):
     return packed, scales, x_new
 
 
-@pytest.mark.parametrize("d,group", [(64, 32), (64, 64), (128, 32), (128, 128), (256, 64),
-                                     (256, 256)])
-@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
-@pytest.mark.parametrize("heads,cap,pos", [(1, 1, 0), (2, 40, 0), (2, 40, 17), (3, 64, 63),
-                                           (5, 300, 257), (52, 70, 33)])
-def test_decode_matches_separate_kernels_and_oracle(kvq, d, group, rot, heads, cap, pos):
+WIDE_MAX_ROWS = 1 << 16  # calls with more rows run the tiled kernel
+
+
+def run_and_check(kvq, d, group, rot, heads, cap, pos, seed):
     signs_np = W.make_signs(d)
     signs = torch.from_numpy(signs_np).cuda()
-    packed, scales, x_new = make_cache(kvq, heads, cap, pos, d, group, rot, signs,
-                                       seed=d + 7 * pos + heads)
+    packed, scales, x_new = make_cache(kvq, heads, cap, pos, d, group, rot, signs, seed)
     before_p, before_s = packed.clone(), scales.clone()
     out = kvq.kvq_decode_step(x_new, packed, scales, pos, signs, rot, group)
     torch.cuda.synchronize()
@@ -57,25 +54,45 @@ def test_decode_matches_separate_kernels_and_oracle(kvq, d, group, rot, heads, c
     keep[pos] = False
     assert torch.equal(packed[:, keep], before_p[:, keep])
     assert torch.equal(scales[:, keep], before_s[:, keep])
-    # row pos == forward kernel on x_new, bit for bit
     p_new, s_new = kvq.kvq_rot_quant_fwd(x_new, signs, rot, group)
-    assert torch.equal(packed[:, pos], p_new)
-    assert torch.equal(scales[:, pos], s_new)
-    # out == inverse kernel on rows [0, pos], bit for bit
     rows_p = packed[:, : pos + 1].reshape(-1, d // 2).contiguous()
     rows_s = scales[:, : pos + 1].reshape(-1, d // group).contiguous()
     ref = kvq.kvq_dequant_rot_inv(rows_p, rows_s, signs, rot, group).reshape(heads, pos + 1, d)
-    assert torch.equal(out, ref)
-    # oracle: the new row's codes/scales and the whole output
     xn = x_new.cpu().numpy()
-    check_fwd(xn, signs_np, rot, group, p_new.cpu().numpy(), s_new.cpu().numpy())
+    if heads * (pos + 1) > WIDE_MAX_ROWS:
+        # tiled kernel: same arithmetic as the forward / inverse kernels
+        assert torch.equal(packed[:, pos], p_new)
+        assert torch.equal(scales[:, pos], s_new)
+        assert torch.equal(out, ref)
+    # new row against the oracle (codes, scales) and its output row
+    check_fwd(xn, signs_np, rot, group, packed[:, pos].cpu().numpy(),
+              scales[:, pos].cpu().numpy(), max_flip_fraction=None)
     o = out.cpu().numpy()
+    check_inv(xn, signs_np, rot, group, packed[:, pos].cpu().numpy(),
+              scales[:, pos].cpu().numpy(), o[:, pos], None)
+    # every row against the oracle inverse of the stored codes and scales
     ref_o = O.dequant_rot_inv(rows_p.cpu().numpy(), rows_s.cpu().numpy(), signs_np, rot,
-                              group).reshape(heads, pos + 1, d)
-    tol = 2e-3 * np.abs(ref_o.astype(np.float64)).max(axis=2, keepdims=True) + 1e-6
-    assert np.all(np.abs(o.astype(np.float64) - ref_o.astype(np.float64)) <= tol)
-    check_inv(xn, signs_np, rot, group, p_new.cpu().numpy(), s_new.cpu().numpy(),
-              o[:, pos], None)
+                              group).reshape(heads, pos + 1, d).astype(np.float64)
+    tol = 2e-3 * np.abs(ref_o).max(axis=2, keepdims=True) + 1e-6
+    assert np.all(np.abs(o.astype(np.float64) - ref_o) <= tol)
+    # and against the inverse kernel on the same rows
+    assert np.all(np.abs(o.astype(np.float64) - ref.cpu().numpy().astype(np.float64)) <= tol)
+
+
+@pytest.mark.parametrize("d,group", [(64, 32), (64, 64), (128, 32), (128, 128), (256, 64),
+                                     (256, 256), (256, 32), (128, 64)])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("heads,cap,pos", [(1, 1, 0), (2, 40, 0), (2, 40, 17), (3, 64, 63),
+                                           (5, 300, 257), (52, 70, 33)])
+def test_decode_small_calls(kvq, d, group, rot, heads, cap, pos):
+    run_and_check(kvq, d, group, rot, heads, cap, pos, seed=d + 7 * pos + heads)
+
+
+@pytest.mark.parametrize("d,group", [(64, 64), (128, 32), (256, 256)])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+def test_decode_large_call_tiled(kvq, d, group, rot):
+    """More than 2^16 rows: the tiled kernel, bit-identical to fwd / inv."""
+    run_and_check(kvq, d, group, rot, heads=3, cap=23000, pos=22001, seed=d + rot)
 
 
 def test_gemma_decode_steps(kvq):
