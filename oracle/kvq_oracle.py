@@ -26,7 +26,7 @@ transforms.  Every function cites the passage it follows.  Sources:
   "Python: Quantize, Simulate the Integer GEMM...": qmax = 2**(b-1)-1,
   scale = amax/qmax, q = clamp(round(x/scale), -qmax-1, qmax).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * R1 real packing of the rfft output into d reals (stated with the problem):
   y[0] = Re X_0/sqrt(d), y[1] = Re X_{d/2}/sqrt(d),

@@ -603,13 +603,12 @@ __device__ __noinline__ void drain_and_fail(uint32_t bars, const Ring& r, unsign
   atomicOr(status, 1u);
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int MINB>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                    const FwdArgs a, unsigned* status) {
   using C = Cfg<D, ROT, TPV>;
   using Gr = Groups<C, G>;
-  constexpr int S_OUT = 2;
   constexpr int WARP_BYTES = S_IN * C::XTILE + S_OUT * C::QTILE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
@@ -696,13 +695,12 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int MINB>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_inv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmX, const InvArgs a, unsigned* status) {
   using C = Cfg<D, ROT, TPV>;
   using Gr = Groups<C, G>;
-  constexpr int S_OUT = 2;
   constexpr int STILE = C::VPW * Gr::NG * 4;
   constexpr int STAGE = C::QTILE + ((STILE + 1023) / 1024) * 1024;
   constexpr int WARP_BYTES = S_IN * STAGE + S_OUT * C::XTILE;
@@ -962,10 +960,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
 }
 
 // Dynamic shared memory each kernel needs (plus 1 KiB alignment slack).
-template <int D, int ROT, int TPV, int S_IN>
+template <int D, int ROT, int TPV, int S_IN, int S_OUT>
 constexpr int fwd_smem_bytes() {
   using C = Cfg<D, ROT, TPV>;
-  return kWarps * (S_IN * C::XTILE + 2 * C::QTILE) + 1024;
+  return kWarps * (S_IN * C::XTILE + S_OUT * C::QTILE) + 1024;
 }
 
 template <int D, int ROT, int TPV, int S_IN>
@@ -974,12 +972,12 @@ constexpr int decode_smem_bytes() {
   return kWarps * (S_IN * C::QTILE + 2 * C::XTILE) + 1024;
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT>
 constexpr int inv_smem_bytes() {
   using C = Cfg<D, ROT, TPV>;
   constexpr int STILE = C::VPW * (D / G) * 4;
   constexpr int STAGE = C::QTILE + ((STILE + 1023) / 1024) * 1024;
-  return kWarps * (S_IN * STAGE + 2 * C::XTILE) + 1024;
+  return kWarps * (S_IN * STAGE + S_OUT * C::XTILE) + 1024;
 }
 
 }  // namespace kvq

@@ -17,39 +17,31 @@ namespace kvq {
 // Bit 0: a bounded wait on an asynchronous copy ran out.
 static __device__ unsigned g_status;
 
-// Per-d launch tuning: pipeline depth (tiles in flight per warp) and the
-// minimum resident blocks per SM the register allocation must allow.
-#ifndef KVQ_FWD_MINB_64
-#define KVQ_FWD_MINB_64 4
-#endif
-#ifndef KVQ_INV_MINB_64
-#define KVQ_INV_MINB_64 4
-#endif
-#ifndef KVQ_FWD_MINB_128
-#define KVQ_FWD_MINB_128 2
-#endif
-#ifndef KVQ_INV_MINB_128
-#define KVQ_INV_MINB_128 2
-#endif
-#ifndef KVQ_FWD_MINB_256
-#define KVQ_FWD_MINB_256 2
-#endif
-#ifndef KVQ_INV_MINB_256
-#define KVQ_INV_MINB_256 2
-#endif
+// Per-(d, rotation, direction) launch tuning: pipeline depth (tiles in
+// flight per warp), output tiles in flight, and the minimum resident blocks
+// per SM the register allocation must allow.  Chosen from same-box sweeps on
+// the B200: the SRFT kernels at d = 256 are issue-bound, so fewer resident
+// warps with more registers each win for the forward direction, while the
+// inverse gains from a third block despite an 8-byte spill.
 #ifndef KVQ_INV_STAGES_64
 #define KVQ_INV_STAGES_64 2
 #endif
+#ifndef KVQ_INV_STAGES_BIG
+#define KVQ_INV_STAGES_BIG 2
+#endif
+#ifndef KVQ_SOUT_BIG
+#define KVQ_SOUT_BIG 1
+#endif
 
-template <int D>
+template <int D, int ROT>
 struct Tuning {
   static constexpr int TPV = DefaultTPV<D>::value;
   static constexpr int FWD_STAGES = 2;
-  static constexpr int INV_STAGES = D == 64 ? KVQ_INV_STAGES_64 : 3;
-  static constexpr int FWD_MINB =
-      D == 64 ? KVQ_FWD_MINB_64 : (D == 128 ? KVQ_FWD_MINB_128 : KVQ_FWD_MINB_256);
-  static constexpr int INV_MINB =
-      D == 64 ? KVQ_INV_MINB_64 : (D == 128 ? KVQ_INV_MINB_128 : KVQ_INV_MINB_256);
+  static constexpr int INV_STAGES = D == 64 ? KVQ_INV_STAGES_64 : KVQ_INV_STAGES_BIG;
+  static constexpr int S_OUT = D == 64 ? 2 : KVQ_SOUT_BIG;
+  static constexpr bool SRFT = ROT == kRotSRFT;
+  static constexpr int FWD_MINB = D == 64 ? 4 : (D == 128 ? 3 : (SRFT ? 2 : 3));
+  static constexpr int INV_MINB = D == 64 ? 4 : (D == 128 ? (SRFT ? 3 : 2) : 3);
 };
 
 namespace detail {
@@ -109,9 +101,9 @@ inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
 
 template <int D, int G, int ROT>
 cudaError_t fwd_one(const FwdLaunch& L) {
-  using T = Tuning<D>;
-  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::FWD_MINB>;
-  constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES>();
+  using T = Tuning<D, ROT>;
+  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, T::FWD_MINB>;
+  constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES, T::S_OUT>();
   int occ;
   unsigned* st;
   cudaError_t e = setup<kern>(smem, &occ);
@@ -125,9 +117,9 @@ cudaError_t fwd_one(const FwdLaunch& L) {
 
 template <int D, int G, int ROT>
 cudaError_t inv_one(const InvLaunch& L) {
-  using T = Tuning<D>;
-  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::INV_MINB>;
-  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES>();
+  using T = Tuning<D, ROT>;
+  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB>;
+  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT>();
   int occ;
   unsigned* st;
   cudaError_t e = setup<kern>(smem, &occ);
@@ -142,7 +134,7 @@ cudaError_t inv_one(const InvLaunch& L) {
 
 template <int D, int G, int ROT>
 cudaError_t decode_one(const DecodeLaunch& L) {
-  using T = Tuning<D>;
+  using T = Tuning<D, ROT>;
   constexpr auto kern = kvq_decode_kernel<D, G, ROT, T::TPV, T::INV_STAGES, 1>;
   constexpr int smem = decode_smem_bytes<D, ROT, T::TPV, T::INV_STAGES>();
   int occ;
