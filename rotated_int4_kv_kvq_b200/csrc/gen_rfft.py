@@ -2,14 +2,16 @@
 
     python rotated_int4_kv_kvq_b200/csrc/gen_rfft.py
 
-For n in {64, 128} it emits
+For n in {32, 64} it emits two-lane codelets over f2 values (two
+independent transforms in lock step, one per lane of each packed fp32x2
+register):
 
-  rfft<n>(x, y):  y[0] = X_0/sqrt2, y[1] = X_{n/2}/sqrt2,
-                  y[2k] = Re X_k, y[2k+1] = Im X_k   (1 <= k < n/2),
-                  X_k = sum_m x_m exp(-2 pi i k m / n)  (unnormalized);
-  irfft<n>(y, x): the transpose map, x_m = sum_k X_k exp(+2 pi i k m / n)
-                  with X rebuilt from y in the same packing (X_0 = sqrt2 y[0],
-                  X_{n/2} = sqrt2 y[1]).
+  rfft<n>x2_fwd(x, y):  y[0] = X_0/sqrt2, y[1] = X_{n/2}/sqrt2,
+                        y[2k] = Re X_k, y[2k+1] = Im X_k   (1 <= k < n/2),
+                        X_k = sum_m x_m exp(-2 pi i k m / n)  (unnormalized);
+  rfft<n>x2_inv(y, x):  the transpose map, x_m = sum_k X_k exp(+2 pi i k m / n)
+                        with X rebuilt from y in the same packing (X_0 =
+                        sqrt2 y[0], X_{n/2} = sqrt2 y[1]).
 
 The transforms follow the split-radix decomposition for real data (even
 samples through a half-length real DFT, samples 4m+1 and 4m+3 through two
@@ -17,9 +19,10 @@ quarter-length real DFTs, recombined with twiddles W^k and W^3k), keeping
 only the non-redundant half of every Hermitian spectrum.  The generator
 builds an expression graph with hash-consing, folds trivial twiddles
 (+-1, +-i) and negations into add/sub, writes twiddle products as fused
-multiply-adds, and checks the graph numerically against numpy's FFT before
-emitting anything.  Twiddle constants are cos/sin evaluated in double and
-rounded once to float.
+multiply-adds, checks the graph numerically against numpy's FFT, then
+checks the emitted instruction list (with the polarity of every output, see
+emit_x2) against the graph before writing anything.  Twiddle constants are
+cos/sin evaluated in double and rounded once to float.
 """
 
 from __future__ import annotations
@@ -318,70 +321,143 @@ def use_counts(g: Graph, outs, live):
     return uses
 
 
-def emit(name, g: Graph, outs, in_arr, out_arr, n):
-    """Straight-line code; an add/sub whose operand is a product used only
-    there is emitted as one fused multiply-add."""
+def emit_x2(name, g: Graph, outs, in_arr, out_arr, n):
+    """Two-lane version of `emit`: every value is an f2 (two independent
+    transforms in lock step, constants broadcast to both lanes), built only
+    from add/sub/mul/fma.rn.f32x2, which take no negated operands.  Each
+    emitted value therefore carries a polarity p (the register holds p times
+    the true value), chosen per operation so that one instruction suffices;
+    the polarity of every output is returned for the caller to absorb.
+    Returns (code, op count, output polarities, op list for `run_x2`)."""
     live = live_nodes(g, outs)
     uses = use_counts(g, outs, live)
-    fused = {}  # add/sub node -> (mul operand index, other operand, sign of other)
+    fused = {}
     absorbed = set()
     for i in sorted(live):
         op, args = g.nodes[i]
         if op not in ("add", "sub"):
             continue
-        for pos in (1, 0) if op == "add" else (1, 0):
+        for pos in (1, 0):
             m = args[pos]
             mop, margs = g.nodes[m]
             if mop == "mul" and uses[m] == 1 and m not in absorbed:
                 other = args[1 - pos]
-                # add: m + other; sub: args[0] - args[1]
                 if op == "add":
                     fused[i] = (m, +1, other, +1)
-                elif pos == 1:  # other - m
+                elif pos == 1:
                     fused[i] = (m, -1, other, +1)
-                else:  # m - other
+                else:
                     fused[i] = (m, +1, other, -1)
                 absorbed.add(m)
                 break
-    lines = [f"__device__ __forceinline__ void {name}(const float (&{in_arr})[{n}], "
-             f"float (&{out_arr})[{n}]) {{"]
-    counts = {"add": 0, "sub": 0, "mul": 0, "fma": 0}
+    pol = {}
+    prog = []  # (dst, op, a, b, const): op in add/sub/mul/fma; fma = a*const + b
+    lines = [f"__device__ __forceinline__ void {name}(const f2 (&{in_arr})[{n}], "
+             f"f2 (&{out_arr})[{n}]) {{"]
 
     def ref(i):
         op, args = g.nodes[i]
         return args[0] if op == "in" else f"t{i}"
 
+    def lin(i, a, ca, b, cb):
+        """value = ca*a + cb*b (ca a constant, cb = +-1) as one fma."""
+        cb_eff = cb * pol[b]
+        c_eff = ca * pol[a]
+        if cb_eff > 0:
+            return ("fma", a, b, c_eff, +1)
+        return ("fma", a, b, -c_eff, -1)
+
+    counts = {"add": 0, "sub": 0, "mul": 0, "fma": 0}
     for i, (op, args) in enumerate(g.nodes):
-        if i not in live or op == "in" or i in absorbed:
+        if i not in live or i in absorbed:
+            continue
+        if op == "in":
+            pol[i] = +1
             continue
         if i in fused:
             m, msign, other, osign = fused[i]
             src, c = g.nodes[m][1]
-            e = f"fmaf({ref(src)}, {fmt(msign * c)}, {'-' if osign < 0 else ''}{ref(other)})"
-            counts["fma"] += 1
-        elif op == "add":
-            e = f"{ref(args[0])} + {ref(args[1])}"
-            counts["add"] += 1
-        elif op == "sub":
-            e = f"{ref(args[0])} - {ref(args[1])}"
-            counts["sub"] += 1
+            kind, a, b, cc, p = lin(i, src, msign * c, other, osign)
+        elif op == "fma":
+            kind, a, b, cc, p = lin(i, args[0], args[1], args[2], +1)
         elif op == "mul":
-            e = f"{ref(args[0])} * {fmt(args[1])}"
-            counts["mul"] += 1
+            kind, a, b, cc, p = "mul", args[0], None, args[1] * pol[args[0]], +1
         else:
-            e = f"fmaf({ref(args[0])}, {fmt(args[1])}, {ref(args[2])})"
-            counts["fma"] += 1
-        lines.append(f"  const float t{i} = {e};")
+            x, y = args
+            sy = +1 if op == "add" else -1
+            px, py = pol[x], pol[y] * sy  # value = px*X' + py*Y'
+            if px > 0 and py > 0:
+                kind, a, b, p = "add", x, y, +1
+            elif px > 0:
+                kind, a, b, p = "sub", x, y, +1
+            elif py > 0:
+                kind, a, b, p = "sub", y, x, +1
+            else:
+                kind, a, b, p = "add", x, y, -1
+            cc = None
+        pol[i] = p
+        prog.append((i, kind, a, b, cc))
+        counts[kind] += 1
+        if kind == "add":
+            e = f"add2({ref(a)}, {ref(b)})"
+        elif kind == "sub":
+            e = f"sub2({ref(a)}, {ref(b)})"
+        elif kind == "mul":
+            e = f"mul2({ref(a)}, mk2({fmt(cc)}, {fmt(cc)}))"
+        else:
+            e = f"fma2({ref(a)}, mk2({fmt(cc)}, {fmt(cc)}), {ref(b)})"
+        lines.append(f"  const f2 t{i} = {e};")
+    opol = []
     for j, o in enumerate(outs):
         if o.node is None:
-            lines.append(f"  {out_arr}[{j}] = 0.0f;")
+            lines.append(f"  {out_arr}[{j}] = mk2(0.0f, 0.0f);")
+            opol.append(+1)
         else:
-            lines.append(f"  {out_arr}[{j}] = {'-' if o.sign < 0 else ''}{ref(o.node)};")
+            lines.append(f"  {out_arr}[{j}] = {ref(o.node)};")
+            opol.append(o.sign * pol[o.node])
     lines.append("}")
     total = sum(counts.values())
     head = (f"// {name}: {counts['add'] + counts['sub']} add/sub, {counts['mul']} mul, "
-            f"{counts['fma']} fma ({total} fp32 instructions)")
-    return head + "\n" + "\n".join(lines) + "\n", total
+            f"{counts['fma']} fma ({total} f32x2 instructions)")
+    outs_nodes = [o.node for o in outs]
+    return head + "\n" + "\n".join(lines) + "\n", total, opol, (prog, outs_nodes)
+
+
+def run_x2(g: Graph, prog, outs_nodes, inputs: dict):
+    """Interpret an emit_x2 op list (one lane) on numbers: returns the
+    stored (polarity-scaled) outputs."""
+    vals = {}
+    for i, (op, args) in enumerate(g.nodes):
+        if op == "in":
+            vals[i] = inputs[args[0]]
+    for dst, kind, a, b, cc in prog:
+        if kind == "add":
+            vals[dst] = vals[a] + vals[b]
+        elif kind == "sub":
+            vals[dst] = vals[a] - vals[b]
+        elif kind == "mul":
+            vals[dst] = vals[a] * cc
+        else:
+            vals[dst] = vals[a] * cc + vals[b]
+    return np.array([0.0 if nd is None else vals[nd] for nd in outs_nodes])
+
+
+def check_x2(n, g, outs, prog_outs, opol, forward):
+    """The emitted two-lane program, polarities applied, equals the graph."""
+    rng = np.random.default_rng(100 + n)
+    prog, onodes = prog_outs
+    name = "x" if forward else "y"
+    for _ in range(4):
+        xv = rng.standard_normal(n)
+        inputs = {f"{name}[{i}]": xv[i] for i in range(n)}
+        ref = evaluate(g, outs, inputs)
+        got = run_x2(g, prog, onodes, inputs) * np.array(opol)
+        err = np.abs(got - ref).max() / np.abs(ref).max()
+        assert err < 1e-12, (n, forward, err)
+
+
+def pol_mask(opol):
+    return sum(1 << j for j, p in enumerate(opol) if p < 0)
 
 
 def main(path=None):
@@ -389,25 +465,32 @@ def main(path=None):
     path = path or os.path.join(here, "kvq_rfft.cuh")
     parts = [
         "// kvq_rfft.cuh -- GENERATED by gen_rfft.py; do not edit by hand.\n",
-        "// Real-input split-radix FFT codelets (see gen_rfft.py for the maps).\n",
+        "// Two-lane real-input split-radix FFT codelets (see gen_rfft.py).\n",
         "#pragma once\n\nnamespace kvq {\n\n",
-        "template <int N> struct RFFT;\n\n",
+        "template <int N> struct RFFT2;\n\n",
     ]
-    for n in (64, 128):
+    for n in (32, 64):
         check(n)
         gf, of = build_forward(n)
         gi, oi = build_inverse(n)
-        fwd, cf = emit(f"rfft{n}_fwd", gf, of, "x", "y", n)
-        inv, ci = emit(f"rfft{n}_inv", gi, oi, "y", "x", n)
+        fwd, cf, pf, progf = emit_x2(f"rfft{n}x2_fwd", gf, of, "x", "y", n)
+        inv, ci, pi, progi = emit_x2(f"rfft{n}x2_inv", gi, oi, "y", "x", n)
+        check_x2(n, gf, of, progf, pf, True)
+        check_x2(n, gi, oi, progi, pi, False)
         parts += [fwd, "\n", inv, "\n"]
         parts.append(
-            f"template <> struct RFFT<{n}> {{\n"
-            f"  static __device__ __forceinline__ void fwd(const float (&x)[{n}], float (&y)[{n}]) "
-            f"{{ rfft{n}_fwd(x, y); }}\n"
-            f"  static __device__ __forceinline__ void inv(const float (&y)[{n}], float (&x)[{n}]) "
-            f"{{ rfft{n}_inv(y, x); }}\n"
+            f"// Two independent {n}-point transforms in the two lanes of each f2.\n"
+            f"// Output j holds -1 times its true value where bit j of FWD_NEG / INV_NEG\n"
+            f"// is set.\n"
+            f"template <> struct RFFT2<{n}> {{\n"
+            f"  static constexpr uint64_t FWD_NEG = 0x{pol_mask(pf):016x}ull;\n"
+            f"  static constexpr uint64_t INV_NEG = 0x{pol_mask(pi):016x}ull;\n"
+            f"  static __device__ __forceinline__ void fwd(const f2 (&x)[{n}], f2 (&y)[{n}]) "
+            f"{{ rfft{n}x2_fwd(x, y); }}\n"
+            f"  static __device__ __forceinline__ void inv(const f2 (&y)[{n}], f2 (&x)[{n}]) "
+            f"{{ rfft{n}x2_inv(y, x); }}\n"
             f"}};\n\n")
-        print(f"n={n}: forward {cf} fp32 ops, inverse {ci} fp32 ops", file=sys.stderr)
+        print(f"n={n} x2: forward {cf} f32x2 ops, inverse {ci} f32x2 ops", file=sys.stderr)
     parts.append("}  // namespace kvq\n")
     with open(path, "w") as f:
         f.write("".join(parts))

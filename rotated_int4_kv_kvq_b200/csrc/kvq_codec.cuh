@@ -12,6 +12,10 @@
 //  * Each thread holds its vector (or half of it) in registers and runs the
 //    whole step there: sign flip, rotation (FFT / FWHT, plus one exchange
 //    stage through warp shuffles when TPV = 2), absmax, round, pack.
+//  * SRFT: an fp16 word is an (even, odd) sample pair, so one generated
+//    two-lane real-FFT codelet in packed fp32x2 transforms both parity halves
+//    at once (half the issue slots of a scalar codelet) and a radix-2 join
+//    in scalar fp32 completes the spectrum; the inverse mirrors it.
 //  * Results are written to a shared tile and stored by TMA (bulk groups);
 //    scales are written directly with coalesced vector stores.
 //
@@ -22,12 +26,6 @@
 
 #include "kvq_device.cuh"
 #include "kvq_rfft.cuh"
-
-// Inverse of the one-thread SRFT: 1 = generated c2r codelet, 0 = half-length
-// complex FFT with the real pre-split.
-#ifndef KVQ_INV_CODELET
-#define KVQ_INV_CODELET 0
-#endif
 
 namespace kvq {
 
@@ -40,8 +38,8 @@ constexpr int kThreads = kWarps * 32;
 //  kLayQuarter (SRFT, thread pair):     local half h (E/2 values) of thread t is
 //           quarter qd = h ? 3 - 2t : 2t of y, i.e. thread 0 holds quarters
 //           0 and 3 and thread 1 quarters 2 and 1.  This is where the pair
-//           split of the real FFT leaves each output (see rotate_fwd), and it
-//           makes every (X_k, X_{N-k}) pair but one local to a thread.
+//           join of the two half-length real FFTs leaves each output (see
+//           pair_join_fwd); both halves are in natural y order.
 constexpr int kLayFull = 0, kLayHalf = 1, kLayQuarter = 2;
 
 template <int D_, int ROT_, int TPV_>
@@ -60,15 +58,15 @@ struct Cfg {
   static constexpr int QP = D / 2;         // code row pitch in bytes
   static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
   // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
-  // takes Yin = KAPPA_INV * y_hat.  One-thread SRFT (generated real-FFT
-  // codelets, Y = packed rfft with X_0, X_{d/2} over sqrt2): sqrt(2/d) and
-  // 1/sqrt(2d).  Thread-pair SRFT (Y = 2X packing): 1/sqrt(2d) both ways.
-  // SRHT: 1/sqrt(d) both ways.
+  // takes Yin = KAPPA_INV * y_hat.  SRFT (Y = packed rfft with X_0, X_{d/2}
+  // over sqrt2, from the generated real-FFT codelets, joined across the pair
+  // at d = 256): sqrt(2/d) and 1/sqrt(2d).  SRHT: 1/sqrt(d) both ways.
   static constexpr bool CODELET = ROT == kRotSRFT && TPV == 1;
-  static constexpr bool INV_CODELET = KVQ_INV_CODELET != 0;
+  // Thread-pair SRFT: each thread runs a d/2-point real FFT on the even
+  // (thread 0) or odd (thread 1) samples; one half-volume exchange joins them.
+  static constexpr bool PAIR_RFFT = ROT == kRotSRFT && TPV == 2;
   static constexpr double KAPPA_FWD_D =
-      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D))
-                      : (CODELET ? const_sqrt(2.0 / D) : 1.0 / const_sqrt(2.0 * D));
+      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : const_sqrt(2.0 / D);
   static constexpr double KAPPA_INV_D =
       ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : 1.0 / const_sqrt(2.0 * D);
   static constexpr float KAPPA_INV = float(KAPPA_INV_D);
@@ -81,11 +79,6 @@ struct DefaultTPV {
   static constexpr int value = D >= 256 ? 2 : 1;
 };
 
-// Word (fp16 pair) of the vector held in slot j of thread t.
-template <class C>
-__host__ __device__ constexpr int word_of(int t, int j) {
-  return (C::ROT == kRotSRFT && C::TPV == 2) ? 2 * j + t : t * C::NW + j;
-}
 
 // Quarter of y holding local half h of thread t (kLayQuarter layout).
 __device__ __forceinline__ int quarter_of(int t, int h) { return h ? 3 - 2 * t : 2 * t; }
@@ -102,9 +95,48 @@ __device__ __forceinline__ int global_y(int t, int i) {
   }
 }
 
-template <class C>
+// fp16 sign bits to XOR into word w = (x_{2w}, x_{2w+1}).
 __device__ __forceinline__ uint32_t sign_mask_word(const int8_t* signs, int w) {
   return (signs[2 * w] < 0 ? 0x00008000u : 0u) | (signs[2 * w + 1] < 0 ? 0x80000000u : 0u);
+}
+
+// Sign mask of word j of thread t as load_x hands it out.  Thread-pair SRFT:
+// thread t holds v_m = u_{2m+t} (-1)^{t m}, word j = (v_{2j}, v_{2j+1}); the
+// modulation (-1)^m of thread 1 moves its spectrum by d/4 bins.  Otherwise
+// thread t holds words t*NW + j.
+template <class C>
+__device__ __forceinline__ uint32_t load_mask_word(const int8_t* signs, int t, int j) {
+  if constexpr (C::PAIR_RFFT) {
+    const bool lo = signs[4 * j + t] < 0;
+    const bool hi = (signs[4 * j + 2 + t] < 0) != (t == 1);
+    return (lo ? 0x00008000u : 0u) | (hi ? 0x80000000u : 0u);
+  } else {
+    return sign_mask_word(signs, t * C::NW + j);
+  }
+}
+
+// Sign mask of word j of thread t as store_x receives it (words t*NW + j),
+// including the polarity of the inverse two-lane codelet's outputs.
+// Thread-pair SRFT: the odd samples of every odd word arrive negated (see
+// rotate_inv).
+template <class C>
+__device__ __forceinline__ uint32_t store_mask_word(const int8_t* signs, int t, int j) {
+  uint32_t m = sign_mask_word(signs, t * C::NW + j);
+  if constexpr (C::ROT == kRotSRFT) {
+    constexpr uint64_t neg = RFFT2<C::E / 2>::INV_NEG;  // inverse codelet polarity
+    if constexpr (C::TPV == 1) {
+      if ((neg >> j) & 1u) m ^= 0x80008000u;
+    } else {
+      // word j = 2i + b holds half b of P_i (own) and of P_{i+NR/4}
+      // (partner); thread 1 puts the partner's half first
+      const int i = j / 2;
+      const bool own = (neg >> i) & 1u, other = (neg >> (i + C::NW / 2)) & 1u;
+      const bool lo = t ? other : own, hi = t ? own : other;
+      m ^= (lo ? 0x00008000u : 0u) | (hi ? 0x80000000u : 0u);
+      if (j & 1) m ^= 0x80000000u;
+    }
+  }
+  return m;
 }
 
 // ------------------------------------------------ shared-memory tile I/O ---
@@ -124,7 +156,7 @@ __device__ __forceinline__ uint32_t swq(int row, int c) {
 template <class C>
 __device__ __forceinline__ void load_x(uint32_t tile, int row, int t, uint32_t mask,
                                        uint32_t (&xw)[C::NW]) {
-  if constexpr (C::TPV == 1 || C::ROT == kRotSRHT) {
+  if constexpr (!C::PAIR_RFFT) {
 #pragma unroll
     for (int c = 0; c < C::NW / 4; ++c) {
       const int gc = t * (C::NW / 4) + c;  // chunk of the row
@@ -135,18 +167,23 @@ __device__ __forceinline__ void load_x(uint32_t tile, int row, int t, uint32_t m
       xw[4 * c + 2] = v.z ^ m.z;
       xw[4 * c + 3] = v.w ^ m.w;
     }
-  } else {  // SRFT, TPV = 2: thread t holds the words 2j + t
+  } else {
+    // Both threads of the pair read the whole row; thread t keeps fp16 half
+    // t of every word, two words per result: (u_{4j+t}, u_{4j+2+t}).
+    const uint32_t sel = t ? 0x7632u : 0x5410u;
 #pragma unroll
-    for (int jj = 0; jj < C::NW / 4; ++jj) {
-      const uint4 m = lds128(mask + jj * 16);
-      const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
+    for (int c = 0; c < C::D / 8; ++c) {
+      const uint4 v = lds128(tile + (c / 8) * C::SLAB + sw128(row, c % 8));
+      xw[2 * c] = __byte_perm(v.x, v.y, sel);
+      xw[2 * c + 1] = __byte_perm(v.z, v.w, sel);
+    }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = 4 * jj + r;
-        const int cc = (j % 16) / 2;
-        const uint32_t a = tile + (j / 16) * C::SLAB + sw128(row, cc) + (2 * (j % 2) + t) * 4;
-        xw[j] = lds32(a) ^ mm[r];
-      }
+    for (int c = 0; c < C::NW / 4; ++c) {
+      const uint4 m = lds128(mask + c * 16);
+      xw[4 * c] ^= m.x;
+      xw[4 * c + 1] ^= m.y;
+      xw[4 * c + 2] ^= m.z;
+      xw[4 * c + 3] ^= m.w;
     }
   }
 }
@@ -154,27 +191,12 @@ __device__ __forceinline__ void load_x(uint32_t tile, int row, int t, uint32_t m
 template <class C>
 __device__ __forceinline__ void store_x(uint32_t tile, int row, int t, uint32_t mask,
                                         const uint32_t (&xw)[C::NW]) {
-  if constexpr (C::TPV == 1 || C::ROT == kRotSRHT) {
 #pragma unroll
-    for (int c = 0; c < C::NW / 4; ++c) {
-      const int gc = t * (C::NW / 4) + c;
-      const uint4 m = lds128(mask + c * 16);
-      sts128(tile + (gc / 8) * C::SLAB + sw128(row, gc % 8), xw[4 * c] ^ m.x,
-             xw[4 * c + 1] ^ m.y, xw[4 * c + 2] ^ m.z, xw[4 * c + 3] ^ m.w);
-    }
-  } else {
-#pragma unroll
-    for (int jj = 0; jj < C::NW / 4; ++jj) {
-      const uint4 m = lds128(mask + jj * 16);
-      const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = 4 * jj + r;
-        const int cc = (j % 16) / 2;
-        const uint32_t a = tile + (j / 16) * C::SLAB + sw128(row, cc) + (2 * (j % 2) + t) * 4;
-        sts32(a, xw[j] ^ mm[r]);
-      }
-    }
+  for (int c = 0; c < C::NW / 4; ++c) {
+    const int gc = t * (C::NW / 4) + c;
+    const uint4 m = lds128(mask + c * 16);
+    sts128(tile + (gc / 8) * C::SLAB + sw128(row, gc % 8), xw[4 * c] ^ m.x,
+           xw[4 * c + 1] ^ m.y, xw[4 * c + 2] ^ m.z, xw[4 * c + 3] ^ m.w);
   }
 }
 
@@ -209,6 +231,76 @@ __device__ __forceinline__ void store_codes(uint32_t tile, int row, int t,
 
 constexpr float kSqrt2 = 1.41421356237309504880f;
 
+// Sign of output j of a two-lane codelet (bit j of its polarity mask).
+template <uint64_t NEG, int J>
+__device__ __forceinline__ constexpr float lane_sign() {
+  return ((NEG >> J) & 1u) ? -1.0f : 1.0f;
+}
+
+// In-thread radix-2 join.  y2 is RFFT2<N/2>::fwd of the words of an N-point
+// real sequence, i.e. the packed spectra E (lane x: even samples) and O
+// (lane y: odd samples); Y receives the packed N-point rfft in the codelet
+// packing: Y[0] = (X_0, X_{N/2}) / sqrt2, Y[N/4] = X_{N/4}, and
+// X_k = E_k + W_N^k O_k, X_{N/2-k} = conj(E_k - W_N^k O_k) in Y[k],
+// Y[N/2-k].
+template <int N>
+__device__ __forceinline__ void join_lanes_fwd(const f2 (&y2)[N / 2], f2 (&Y)[N / 2]) {
+  constexpr uint64_t NEG = RFFT2<N / 2>::FWD_NEG;
+  {
+    const float e0 = lane_sign<NEG, 0>() * lo2(y2[0]), o0 = lane_sign<NEG, 0>() * hi2(y2[0]);
+    Y[0] = mk2(e0 + o0, e0 - o0);
+    const float eq = lane_sign<NEG, 1>() * lo2(y2[1]), oq = lane_sign<NEG, 1>() * hi2(y2[1]);
+    Y[N / 4] = mk2(kSqrt2 * eq, -kSqrt2 * oq);  // E - i O at bin N/4
+  }
+  static_for<1, N / 4>([&](auto kk) {
+    constexpr int k = decltype(kk)::value;
+    constexpr float sr = lane_sign<NEG, 2 * k>(), si = lane_sign<NEG, 2 * k + 1>();
+    const float er = sr * lo2(y2[2 * k]), orr = sr * hi2(y2[2 * k]);
+    const float ei = si * lo2(y2[2 * k + 1]), oi = si * hi2(y2[2 * k + 1]);
+    constexpr float c = tw_cos(k, N), s = tw_sin(k, N);
+    const float gr = fmaf(c, orr, s * oi), gi = fmaf(c, oi, -(s * orr));  // W_N^k O_k
+    Y[k] = mk2(er + gr, ei + gi);
+    Y[N / 2 - k] = mk2(er - gr, gi - ei);
+  });
+}
+
+// Thread-pair join of the two half-length real FFTs (d = 2*NR points).
+// On entry y holds this thread's packed NR-point rfft (codelet packing):
+// thread 0 the spectrum E of the even samples, thread 1 the spectrum
+// V_k = O_{k+NR/2} = conj(O_{NR/2-k}) of its modulated odd samples.  The
+// radix-2 step X_k = E_k + W_d^k O_k, X_{NR-k} = conj(E_k - W_d^k O_k) needs
+// one value from the partner per output pair: in step a both threads keep
+// slot a and send slot NR/2 - a.  Thread 0 then forms X_a and X_{NR-a},
+// thread 1 X_{NR/2+a} and X_{NR/2-a} (with W_d^{NR/2-a} O_{NR/2-a} =
+// -i conj(W_d^a V_a)), written to slots a (first quarter of its y) and
+// NR/2 - a (second quarter) of Y.
+template <class C>
+__device__ __forceinline__ void pair_join_fwd(const f2 (&y)[C::D / 4], int t, f2 (&Y)[C::P]) {
+  constexpr int H = C::D / 4;  // slots per thread
+  const bool odd = t != 0;
+  {  // a = 0: slot 0 is (Re, Re) of bins 0 and NR/2
+    const float own = lo2(y[0]);
+    const float r = __shfl_xor_sync(kFull, hi2(y[0]), 1);
+    // thread 0: (X_0, X_d/2)/sqrt2 = (E_0 + O_0, E_0 - O_0)/sqrt2;
+    // thread 1: X_{d/4} = E_{d/4} - i O_{d/4}
+    Y[0] = odd ? mk2(kSqrt2 * r, -kSqrt2 * own) : mk2(own + r, own - r);
+  }
+  static_for<1, H / 2 + 1>([&](auto aa) {
+    constexpr int a = decltype(aa)::value;
+    const float ox = lo2(y[a]), oy = hi2(y[a]);
+    const float rx = __shfl_xor_sync(kFull, lo2(y[H - a]), 1);
+    const float ry = __shfl_xor_sync(kFull, hi2(y[H - a]), 1);
+    // thread 0 twiddles conj(received) = O_a, thread 1 its own V_a
+    const float tx = odd ? ox : rx, ty = odd ? oy : -ry;
+    const float px = odd ? rx : ox, py = odd ? -ry : oy;  // E (thread 1: conj E)
+    constexpr float c = tw_cos(a, C::D), s = tw_sin(a, C::D);
+    const float gx = fmaf(c, tx, s * ty), gy = fmaf(c, ty, -(s * tx));  // W_d^a t
+    const float qx = odd ? gy : gx, qy = odd ? -gx : gy;
+    if constexpr (a < H / 2) Y[a] = mk2(px + qx, py + qy);
+    Y[H - a] = mk2(px - qx, qy - py);
+  });
+}
+
 // Y: this thread's E rotated coordinates as P pairs (local order of the
 // layout), unnormalized: the true y is KAPPA * Y.  Input: sign-flipped fp16
 // words.
@@ -227,85 +319,98 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
 #pragma unroll
       for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
     }
-  } else if constexpr (C::TPV == 1) {
-    // Real-input split-radix codelet: Y = packed rfft of u.
-    float u[C::D], y[C::D];
+  } else {
+    // Each word is (even, odd) sample: one two-lane codelet transforms both
+    // parity halves of this thread's E samples, the join makes their rfft.
+    f2 u[C::NW], y2[C::NW];
 #pragma unroll
     for (int j = 0; j < C::NW; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
-      u[2 * j] = f.x;
-      u[2 * j + 1] = f.y;
+      u[j] = mk2(f.x, f.y);
     }
-    RFFT<C::D>::fwd(u, y);
-#pragma unroll
-    for (int k = 0; k < C::P; ++k) Y[k] = mk2(y[2 * k], y[2 * k + 1]);
-  } else {
-    // Thread pair, d/2 = N complex points, M = N/2 per thread, Q = M/2.
-    // Thread t holds z_{2m+t}: in-thread FFT_M gives F_t(k); thread 1 turns
-    // F_1(k) into G(k) = W_N^k F_1(k); one exchange gives, per slot k,
-    //   k <  Q: thread 0 Z_k = F0 + G,        thread 1 Z_{k+M} = F0 - G,
-    //   k >= Q: thread 0 Z_{k+M} = F0 - G,    thread 1 Z_k = F0 + G,
-    // so that both threads pair slot k with slot M - k for the real split
-    // (only the pair (Q, Q) straddles the threads).
-    constexpr int M = C::D / 4;
-    constexpr int N = C::D / 2;
-    constexpr int Q = M / 2;
-    constexpr int LM = ilog2(M);
-    f2 z[M];
-#pragma unroll
-    for (int j = 0; j < M; ++j) {
-      const float2 f = half2_bits_to_float2(xw[j]);
-      z[j] = mk2(f.x, f.y);
-    }
-    fft_dif<M, false>(z);
-    const float sg = t ? -1.0f : 1.0f;
-    const f2 sgA = mk2(sg, sg), sgB = mk2(-sg, -sg);
-    static_for<0, M>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      constexpr int sl = bitrev(k, LM);
-      f2 own = z[sl];
-      if constexpr (k != 0) {
-        if (t) own = twiddle<N, k, false>(own);
-      }
-      const f2 p = shfl_xor2(own, 1);
-      z[sl] = (k < Q) ? fma2(sgA, own, p) : fma2(sgB, p, own);
-    });
-    {  // slot 0: thread 0 Z_0 -> sqrt2 X_0, sqrt2 X_{d/2}; thread 1 Z_M -> 2 conj Z_M
-      const float a = lo2(z[0]), b = hi2(z[0]);
-      Y[0] = t ? mk2(2.0f * a, -2.0f * b) : mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
-    }
-    static_for<1, Q>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      const f2 p1 = add2(z[bitrev(k, LM)], z[bitrev(M - k, LM)]);
-      const f2 p2 = sub2(z[bitrev(k, LM)], z[bitrev(M - k, LM)]);
-      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
-      // thread 0: W_d^k (-i T); thread 1 holds Z_{k+M}: W_d^{k+M} = -i W_d^k,
-      // so it applies W_d^k to (-T).
-      const float pr = t ? -tr : ti, pi = t ? -ti : -tr;
-      constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float wr = fmaf(c, pr, s * pi), wi = fmaf(c, pi, -(s * pr));
-      Y[k] = mk2(sr + wr, si + wi);
-      Y[M - k] = mk2(sr - wr, wi - si);
-    });
-    {  // slot Q: partner across the pair; thread 0 makes X_{Q+M}, thread 1 X_Q
-      const f2 own = z[bitrev(Q, LM)];
-      const f2 other = shfl_xor2(own, 1);
-      const f2 p1 = add2(own, other), p2 = sub2(own, other);
-      const float sr = lo2(p1), ti = hi2(p1), tr = lo2(p2), si = hi2(p2);
-      const float pr = t ? ti : -tr, pi = t ? -tr : -ti;
-      constexpr float c = tw_cos(Q, C::D), s = tw_sin(Q, C::D);
-      const float wr = fmaf(c, pr, s * pi), wi = fmaf(c, pi, -(s * pr));
-      Y[Q] = mk2(sr + wr, si + wi);
+    RFFT2<C::E / 2>::fwd(u, y2);
+    if constexpr (C::TPV == 1) {
+      join_lanes_fwd<C::E>(y2, Y);
+    } else {
+      f2 yt[C::P];
+      join_lanes_fwd<C::E>(y2, yt);
+      pair_join_fwd<C>(yt, t, Y);
     }
   }
 }
 
 // ------------------------------------------------------ inverse rotation ---
 
+// Inverse of join_lanes_fwd: from the packed N-point spectrum Y build the
+// two-lane input of RFFT2<N/2>::inv, z = (E'', O'') with
+// E''_k = X_k + conj X_{N/2-k} and O''_k = W_N^{-k} (X_k - conj X_{N/2-k}),
+// so that lane x of the inverse is the unnormalized N-point inverse at the
+// even samples and lane y at the odd samples.
+template <int N>
+__device__ __forceinline__ void split_lanes_inv(const f2 (&Y)[N / 2], f2 (&z)[N / 2]) {
+  {
+    const float a = lo2(Y[0]), b = hi2(Y[0]);
+    z[0] = mk2(a + b, a - b);
+    z[1] = mk2(kSqrt2 * lo2(Y[N / 4]), -kSqrt2 * hi2(Y[N / 4]));
+  }
+  static_for<1, N / 4>([&](auto kk) {
+    constexpr int k = decltype(kk)::value;
+    const float xr = lo2(Y[k]), xi = hi2(Y[k]);
+    const float mr = lo2(Y[N / 2 - k]), mi = hi2(Y[N / 2 - k]);
+    const float dr = xr - mr, di = xi + mi;
+    constexpr float c = tw_cos(k, N), s = tw_sin(k, N);
+    z[2 * k] = mk2(xr + mr, fmaf(c, dr, -(s * di)));
+    z[2 * k + 1] = mk2(xi - mi, fmaf(c, di, s * dr));
+  });
+}
+
+// Inverse of pair_join_fwd, up to a factor 2 folded into KAPPA_INV: from the
+// two quarters of y_hat this thread holds, rebuild its half-length spectrum
+// (thread 0: E; thread 1: V, additionally multiplied by (-1)^k so that its
+// inverse FFT comes out rotated by NR/2 samples, see rotate_inv).  In step a
+// both threads form S = h0 + conj(h1) and D = h0 - conj(h1) from their pair
+// (h0, h1); thread 0 keeps E_a = S and sends conj(O_a) = W_d^a conj(D),
+// thread 1 keeps i conj(W_d^a conj(D)) and sends conj(S) = E_{NR/2-a}.
+template <class C>
+__device__ __forceinline__ void pair_join_inv(const f2 (&Y)[C::P], int t, f2 (&Z)[C::D / 4]) {
+  constexpr int H = C::D / 4;
+  const bool odd = t != 0;
+  {  // a = 0
+    const float hx = lo2(Y[0]), hy = hi2(Y[0]);
+    const float keep = odd ? -kSqrt2 * hy : hx + hy;
+    const float send = odd ? kSqrt2 * hx : hx - hy;
+    Z[0] = mk2(keep, __shfl_xor_sync(kFull, send, 1));
+  }
+  static_for<1, H / 2 + 1>([&](auto aa) {
+    constexpr int a = decltype(aa)::value;
+    const float h1x = lo2(Y[H - a]), h1y = hi2(Y[H - a]);
+    float h0x, h0y;
+    if constexpr (a < H / 2) {
+      h0x = lo2(Y[a]);
+      h0y = hi2(Y[a]);
+    } else {  // the pair of slot NR/4 straddles the threads
+      h0x = __shfl_xor_sync(kFull, h1x, 1);
+      h0y = __shfl_xor_sync(kFull, h1y, 1);
+    }
+    const float sx = h0x + h1x, sy = h0y - h1y;
+    const float dx = h0x - h1x, dy = h0y + h1y;
+    constexpr float sg = (a & 1) ? -1.0f : 1.0f;  // (-1)^a, thread 1's rotation
+    constexpr float c = sg * tw_cos(a, C::D), s = sg * tw_sin(a, C::D);
+    const float mx = fmaf(c, dx, -(s * dy)), my = -fmaf(c, dy, s * dx);
+    const float kx = odd ? my : sx, ky = odd ? mx : sy;
+    if constexpr (a < H / 2) {
+      const float ex = odd ? sx : mx, ey = odd ? -sy : my;
+      Z[H - a] = mk2(__shfl_xor_sync(kFull, ex, 1), __shfl_xor_sync(kFull, ey, 1));
+    }
+    Z[a] = mk2(kx, ky);
+  });
+}
+
 // Thread's fp16 words of u = R^T y_hat.  The input is pre-scaled,
 // Yin = KAPPA * y_hat, so that the unnormalized inverse transform (the exact
 // inverse of rotate_fwd's unnormalized map up to the factor 1/KAPPA^2) yields
-// u itself.
+// u itself.  Words of a two-lane codelet output that carry polarity -1 are
+// corrected by the store-side sign mask.
 template <class C>
 __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[C::NW]) {
   if constexpr (C::ROT == kRotSRHT) {
@@ -318,93 +423,35 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     fwht<C::P>(Y);
 #pragma unroll
     for (int j = 0; j < C::NW; ++j) xw[j] = float2_to_half2_bits(lo2(Y[j]), hi2(Y[j]));
-  } else if constexpr (C::TPV == 1 && C::INV_CODELET) {
-    float y[C::D], u[C::D];
-#pragma unroll
-    for (int k = 0; k < C::P; ++k) {
-      y[2 * k] = lo2(Y[k]);
-      y[2 * k + 1] = hi2(Y[k]);
-    }
-    RFFT<C::D>::inv(y, u);
-#pragma unroll
-    for (int n = 0; n < C::NW; ++n) xw[n] = float2_to_half2_bits(u[2 * n], u[2 * n + 1]);
-  } else if constexpr (C::TPV == 1) {
-    // Half-length complex inverse FFT after the real pre-split.
-    constexpr int N = C::D / 2;
-    constexpr int LN = ilog2(N);
-    f2 z[N];
-    {
-      const float a = lo2(Y[0]), b = hi2(Y[0]);
-      z[0] = mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
-    }
-    // Q_k = (A + B) + i W^{-k} (A - B), A = X'_k, B = conj X'_{N-k}
-    static_for<1, N / 2>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      const f2 p1 = add2(Y[k], Y[N - k]);  // (Sr, Di) with B = conj Y[N-k]
-      const f2 p2 = sub2(Y[k], Y[N - k]);  // (Dr, Si)
-      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
-      constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);  // W^{-k} D
-      z[k] = mk2(sr - vi, si + vr);      // S + i V
-      z[N - k] = mk2(sr + vi, vr - si);  // conj(S - i V)
-    });
-    z[N / 2] = mk2(2.0f * lo2(Y[N / 2]), -2.0f * hi2(Y[N / 2]));
-    fft_dif<N, true>(z);
-    static_for<0, N>([&](auto nn) {
-      constexpr int n = decltype(nn)::value;
-      const f2 v = z[bitrev(n, LN)];
-      xw[n] = float2_to_half2_bits(lo2(v), hi2(v));
-    });
   } else {
-    constexpr int M = C::D / 4;
-    constexpr int N = C::D / 2;
-    constexpr int Q = M / 2;
-    constexpr int LM = ilog2(M);
-    f2 z[M];
-    {
-      const float a = lo2(Y[0]), b = hi2(Y[0]);
-      z[0] = t ? mk2(2.0f * a, -2.0f * b) : mk2(kSqrt2 * (a + b), kSqrt2 * (a - b));
+    f2 z[C::NW], x2[C::NW];
+    if constexpr (C::TPV == 1) {
+      split_lanes_inv<C::E>(Y, z);
+    } else {
+      f2 zt[C::D / 4];
+      pair_join_inv<C>(Y, t, zt);
+      split_lanes_inv<C::E>(zt, z);
     }
-    static_for<1, Q>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      const f2 p1 = add2(Y[k], Y[M - k]);
-      const f2 p2 = sub2(Y[k], Y[M - k]);
-      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
-      constexpr float c = tw_cos(k, C::D), s = tw_sin(k, C::D);
-      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);  // W_d^{-k} D
-      // thread 0: Q_k = S + i V, Q_{N-k} = conj(S - i V); thread 1 holds
-      // X'_{k+M}: W_d^{-(k+M)} = i W_d^{-k}, so Q = S - V, conj(S + V).
-      z[k] = t ? mk2(sr - vr, si - vi) : mk2(sr - vi, si + vr);
-      z[M - k] = t ? mk2(sr + vr, -(si + vi)) : mk2(sr + vi, vr - si);
-    });
-    {  // slot Q: thread 0 holds X'_{Q+M}, thread 1 X'_Q; partner across
-      const f2 other = shfl_xor2(Y[Q], 1);
-      const f2 p1 = add2(Y[Q], other), p2 = sub2(Y[Q], other);
-      const float sr = lo2(p1), di = hi2(p1), dr = lo2(p2), si = hi2(p2);
-      constexpr float c = tw_cos(Q, C::D), s = tw_sin(Q, C::D);
-      const float vr = fmaf(c, dr, -(s * di)), vi = fmaf(c, di, s * dr);
-      z[Q] = t ? mk2(sr - vi, si + vr) : mk2(sr - vr, si - vi);
-    }
-    // Inverse of the pair exchange: thread 0 forms E_k = Q_k + Q_{k+M},
-    // thread 1 O_k = (Q_k - Q_{k+M}) W_N^{-k}.
-    const float sg = t ? -1.0f : 1.0f;
-    const f2 sgA = mk2(sg, sg);
-    static_for<0, M>([&](auto kk) {
-      constexpr int k = decltype(kk)::value;
-      const f2 own = z[k];
-      const f2 p = shfl_xor2(own, 1);
-      f2 r = (k < Q) ? fma2(sgA, own, p) : fma2(sgA, p, own);
-      if constexpr (k != 0) {
-        if (t) r = twiddle<N, k, true>(r);
+    RFFT2<C::E / 2>::inv(z, x2);
+    if constexpr (C::TPV == 1) {
+#pragma unroll
+      for (int n = 0; n < C::NW; ++n) xw[n] = float2_to_half2_bits(lo2(x2[n]), hi2(x2[n]));
+    } else {
+      // Thread 0 holds the even samples e_m, thread 1 r_m = (-1)^m o_{m+NR/2}
+      // (o: odd samples), as fp16 pairs P_i = (s_{2i}, s_{2i+1}).  Both keep
+      // P_i and send P_{i+NR/4} (i < NR/4); thread t assembles words
+      // t*NR/2 + 2i, 2i + 1 of x; the odd word's odd sample arrives negated
+      // (fixed by the sign mask).
+      const uint32_t se = t ? 0x1054u : 0x5410u, so = t ? 0x3276u : 0x7632u;
+#pragma unroll
+      for (int i = 0; i < C::NW / 2; ++i) {
+        const uint32_t own = float2_to_half2_bits(lo2(x2[i]), hi2(x2[i]));
+        const f2 v = x2[i + C::NW / 2];
+        const uint32_t r = __shfl_xor_sync(kFull, float2_to_half2_bits(lo2(v), hi2(v)), 1);
+        xw[2 * i] = __byte_perm(own, r, se);
+        xw[2 * i + 1] = __byte_perm(own, r, so);
       }
-      z[k] = r;
-    });
-    fft_dif<M, true>(z);
-    static_for<0, M>([&](auto mm) {
-      constexpr int m = decltype(mm)::value;
-      const f2 v = z[bitrev(m, LM)];
-      xw[m] = float2_to_half2_bits(lo2(v), hi2(v));
-    });
+    }
   }
 }
 
@@ -474,7 +521,7 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const f2 v = Y[g * GP + 4 * w + i];
-        if constexpr (C::CODELET) {  // scalar outputs: no re-pairing moves
+        if constexpr (C::ROT == kRotSRFT) {  // scalar outputs: no re-pairing moves
           f[2 * i] = __float_as_uint(__fmaf_rn(lo2(v), inv, kRoundMagic));
           f[2 * i + 1] = __float_as_uint(__fmaf_rn(hi2(v), inv, kRoundMagic));
         } else {
@@ -536,11 +583,14 @@ struct DecodeArgs {
   int64_t n_tiles;      // n_new_tiles + n_heads * tok_tiles
 };
 
+// s_mask[0, d/2): load-side masks, s_mask[d/2, d): store-side masks, each
+// as NW words per thread role t.
 template <class C>
 __device__ __forceinline__ void fill_sign_masks(const int8_t* signs, uint32_t* s_mask) {
   for (int i = threadIdx.x; i < C::D / 2; i += blockDim.x) {
     const int t = i / C::NW, j = i % C::NW;
-    s_mask[i] = sign_mask_word<C>(signs, word_of<C>(t, j));
+    s_mask[i] = load_mask_word<C>(signs, t, j);
+    s_mask[C::D / 2 + i] = store_mask_word<C>(signs, t, j);
   }
 }
 
@@ -612,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   constexpr int WARP_BYTES = S_IN * C::XTILE + S_OUT * C::QTILE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
-  __shared__ __align__(16) uint32_t s_mask[C::D / 2];
+  __shared__ __align__(16) uint32_t s_mask[C::D];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = C::TPV == 2 ? (lane & 1) : 0;
@@ -706,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   constexpr int WARP_BYTES = S_IN * STAGE + S_OUT * C::XTILE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
-  __shared__ __align__(16) uint32_t s_mask[C::D / 2];
+  __shared__ __align__(16) uint32_t s_mask[C::D];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = C::TPV == 2 ? (lane & 1) : 0;
@@ -727,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     prefetch_tensormap(&tmX);
   }
   __syncthreads();
-  const uint32_t mask = smem_u32(s_mask) + uint32_t(t * C::NW * 4);
+  const uint32_t mask_st = smem_u32(s_mask) + uint32_t((C::D / 2 + t * C::NW) * 4);
 
   const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
   const int64_t nw = int64_t(gridDim.x) * kWarps;
@@ -775,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (lane == 0) bulk_wait_read<S_OUT - 1>();
     __syncwarp();
     const uint32_t xdst = xbuf + uint32_t(o * C::XTILE);
-    store_x<C>(xdst, row, t, mask, xw);
+    store_x<C>(xdst, row, t, mask_st, xw);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -810,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   constexpr int WARP_BYTES = S_IN * STAGE + S_OUT * C::XTILE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN + 1];
-  __shared__ __align__(16) uint32_t s_mask[C::D / 2];
+  __shared__ __align__(16) uint32_t s_mask[C::D];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = C::TPV == 2 ? (lane & 1) : 0;
@@ -828,6 +878,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
   __syncthreads();
   const uint32_t mask = smem_u32(s_mask) + uint32_t(t * C::NW * 4);
+  const uint32_t mask_st = mask + uint32_t(C::D / 2 * 4);
   const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
   const int64_t nw = int64_t(gridDim.x) * kWarps;
 
@@ -868,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     }
     dequantize<C, G>(qw, sc, Y);
     rotate_inv<C>(Y, t, xw);
-    store_x<C>(xout, row, t, mask, xw);
+    store_x<C>(xout, row, t, mask_st, xw);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -942,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (lane == 0) bulk_wait_read<S_OUT - 1>();
     __syncwarp();
     const uint32_t xdst = xbuf + uint32_t(o * C::XTILE);
-    store_x<C>(xdst, row, t, mask, xw);
+    store_x<C>(xdst, row, t, mask_st, xw);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {

@@ -3,9 +3,8 @@
 // * PTX wrappers for mbarriers, TMA tensor copies and bulk-group waits.
 // * Compile-time twiddle factors (cos/sin of 2 pi k / n in double, rounded
 //   once to float) so that every FFT constant is an instruction immediate.
-// * Register-resident transforms: radix-2 decimation-in-frequency complex FFT
-//   (natural-order input, bit-reversed output slots, which are renamed at
-//   compile time) and the Walsh-Hadamard butterfly network.
+// * Packed fp32x2 arithmetic (f2) and the register-resident Walsh-Hadamard
+//   butterfly network; the real FFTs are generated codelets (kvq_rfft.cuh).
 // * int4 quantize / pack and unpack / dequantize on 32-bit words.
 //
 // The method these pieces implement is described in include/kvq.h.
@@ -45,12 +44,6 @@ constexpr int ilog2(int n) {
   int l = 0;
   while ((1 << l) < n) ++l;
   return l;
-}
-
-constexpr int bitrev(int x, int bits) {
-  int r = 0;
-  for (int i = 0; i < bits; ++i) r = (r << 1) | ((x >> i) & 1);
-  return r;
 }
 
 constexpr double kPi = 3.14159265358979323846264338327950288;
@@ -316,53 +309,12 @@ __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
 __device__ __forceinline__ f2 shfl_xor2(f2 a, int m) {
   return mk2(__shfl_xor_sync(kFull, lo2(a), m), __shfl_xor_sync(kFull, hi2(a), m));
 }
-__device__ __forceinline__ f2 sel2(bool c, f2 a, f2 b) { return c ? a : b; }
 
 // max(a, b, c) in one instruction (three-operand max of sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// d * exp(-+ 2 pi i K / N), forward sign for INV = false.
-template <int N, int K, bool INV>
-__device__ __forceinline__ f2 twiddle(f2 d) {
-  if constexpr (K % N == 0) {
-    return d;
-  } else if constexpr (4 * K == N) {
-    const float x = lo2(d), y = hi2(d);
-    return INV ? mk2(-y, x) : mk2(y, -x);  // * (+i) : * (-i)
-  } else {
-    constexpr float c = tw_cos(K, N);
-    constexpr float s = tw_sin(K, N);
-    const float x = lo2(d), y = hi2(d);
-    if constexpr (!INV) {  // * (c - i s)
-      return mk2(fmaf(x, c, y * s), fmaf(y, c, -(x * s)));
-    } else {  // * (c + i s)
-      return mk2(fmaf(x, c, -(y * s)), fmaf(y, c, x * s));
-    }
-  }
-}
-
-// In-place radix-2 DIF FFT of length N over complex registers,
-// X_k = sum_n z_n exp(-+ 2 pi i k n / N) (no normalization).  Input in
-// natural order; X_k ends in slot bitrev(k).
-template <int N, bool INV>
-__device__ __forceinline__ void fft_dif(f2 (&z)[N]) {
-  constexpr int L = ilog2(N);
-  static_for<0, L>([&](auto st) {
-    constexpr int h = N >> (decltype(st)::value + 1);
-    static_for<0, N / 2>([&](auto b) {
-      constexpr int bb = decltype(b)::value;
-      constexpr int o = bb % h;
-      constexpr int i = (bb / h) * 2 * h + o;
-      constexpr int j = i + h;
-      const f2 a = z[i], c = z[j];
-      z[i] = add2(a, c);
-      z[j] = twiddle<2 * h, o, INV>(sub2(a, c));
-    });
-  });
 }
 
 // In-place unnormalized Walsh-Hadamard transform (Sylvester order) of the

@@ -20,9 +20,8 @@ static __device__ unsigned g_status;
 // Per-(d, rotation, direction) launch tuning: pipeline depth (tiles in
 // flight per warp), output tiles in flight, and the minimum resident blocks
 // per SM the register allocation must allow.  Chosen from same-box sweeps on
-// the B200: the SRFT kernels at d = 256 are issue-bound, so fewer resident
-// warps with more registers each win for the forward direction, while the
-// inverse gains from a third block despite an 8-byte spill.
+// the B200 (the d = 256 SRFT inverse keeps a third block despite a small
+// spill: it measured faster than two blocks without one).
 #ifndef KVQ_INV_STAGES_64
 #define KVQ_INV_STAGES_64 2
 #endif
@@ -32,6 +31,21 @@ static __device__ unsigned g_status;
 #ifndef KVQ_SOUT_BIG
 #define KVQ_SOUT_BIG 1
 #endif
+#ifndef KVQ_FWD_MINB_64
+#define KVQ_FWD_MINB_64 4
+#endif
+#ifndef KVQ_INV_MINB_64
+#define KVQ_INV_MINB_64 4
+#endif
+#ifndef KVQ_MINB_128_SRFT
+#define KVQ_MINB_128_SRFT 3
+#endif
+#ifndef KVQ_FWD_MINB_256_SRFT
+#define KVQ_FWD_MINB_256_SRFT 3
+#endif
+#ifndef KVQ_INV_MINB_256_SRFT
+#define KVQ_INV_MINB_256_SRFT 3
+#endif
 
 template <int D, int ROT>
 struct Tuning {
@@ -40,8 +54,12 @@ struct Tuning {
   static constexpr int INV_STAGES = D == 64 ? KVQ_INV_STAGES_64 : KVQ_INV_STAGES_BIG;
   static constexpr int S_OUT = D == 64 ? 2 : KVQ_SOUT_BIG;
   static constexpr bool SRFT = ROT == kRotSRFT;
-  static constexpr int FWD_MINB = D == 64 ? 4 : (D == 128 ? 3 : (SRFT ? 2 : 3));
-  static constexpr int INV_MINB = D == 64 ? 4 : (D == 128 ? (SRFT ? 3 : 2) : 3);
+  static constexpr int FWD_MINB =
+      D == 64 ? KVQ_FWD_MINB_64 : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 3)
+                                        : (SRFT ? KVQ_FWD_MINB_256_SRFT : 3));
+  static constexpr int INV_MINB =
+      D == 64 ? KVQ_INV_MINB_64 : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 2)
+                                        : (SRFT ? KVQ_INV_MINB_256_SRFT : 3));
 };
 
 namespace detail {
