@@ -521,7 +521,7 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const f2 v = Y[g * GP + 4 * w + i];
-        if constexpr (C::ROT == kRotSRFT) {  // scalar outputs: no re-pairing moves
+        if constexpr (C::ROT == kRotSRFT) {  // scalar join outputs: no re-pairing
           f[2 * i] = __float_as_uint(__fmaf_rn(lo2(v), inv, kRoundMagic));
           f[2 * i + 1] = __float_as_uint(__fmaf_rn(hi2(v), inv, kRoundMagic));
         } else {

@@ -32,7 +32,7 @@ static __device__ unsigned g_status;
 #define KVQ_SOUT_BIG 1
 #endif
 #ifndef KVQ_FWD_MINB_64
-#define KVQ_FWD_MINB_64 4
+#define KVQ_FWD_MINB_64 5
 #endif
 #ifndef KVQ_INV_MINB_64
 #define KVQ_INV_MINB_64 4
