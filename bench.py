@@ -598,7 +598,63 @@ def run_suite(kvq, dev):
                                   "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
                                   "algo_bytes_per_step": byts,
                                   "ideal_us": byts / (peak * 1e9) * 1e6})
+    res["decode_windowed"] = run_window_suite(kvq, dev, seq, signs, peak)
     return res
+
+
+def run_window_suite(kvq, dev, seq, signs, peak, window=16):
+    """Gemma-3-1B decode steps with the dequantized-prefix cache: 26 calls
+    per step (one per layer, K and V as 2 heads), timed over the `window`
+    steps of one window (one flush) as a CUDA graph; per-step average."""
+    d, g, L, cap = 256, 256, 26, 4096
+    out = []
+    for rot in (kvq.SRFT, kvq.SRHT):
+        packed = torch.zeros((2 * L, cap, d // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((2 * L, cap, 1), dtype=torch.float32, device=dev)
+        kv = seq.clone()  # the attention view, [52, 4096, 256]
+        for end in (272, 1024, 2048, 4096):
+            first = end - window
+            xs = [[seq[2 * l:2 * l + 2, p].contiguous() for l in range(L)]
+                  for p in range(first, end)]
+
+            def steps():
+                for i, p in enumerate(range(first, end)):
+                    for l in range(L):
+                        kvq.kvq_decode_step_windowed(xs[i][l], packed[2 * l:2 * l + 2],
+                                                     scales[2 * l:2 * l + 2], kv[2 * l:2 * l + 2],
+                                                     p, signs, rot, g, window)
+            for _ in range(2):
+                steps()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            gr = torch.cuda.CUDAGraph()
+            s2 = torch.cuda.Stream()
+            s2.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s2):
+                steps()
+            torch.cuda.current_stream().wait_stream(s2)
+            with torch.cuda.graph(gr):
+                steps()
+            for _ in range(2):
+                gr.replay()
+            torch.cuda.synchronize()
+            reps = 10
+            e0.record()
+            for _ in range(reps):
+                gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / reps / window
+            del gr
+            # per window: every step copies the new rows (2d in, 2d out per
+            # head); the flush re-reads the window and writes codes, scales and
+            # the dequantized rows
+            byts = L * 2 * (window * 4 * d + window * (2 * d + fwd_bytes(d, g)))
+            out.append({"rot": "srft" if rot == 0 else "srht", "pos": end - 1, "window": window,
+                        "graph_us_per_step": us, "algo_bytes_per_step": byts / window,
+                        "ideal_us": byts / window / (peak * 1e9) * 1e6})
+        del packed, scales, kv
+    return out
 
 
 if __name__ == "__main__":

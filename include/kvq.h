@@ -142,6 +142,41 @@ kvq_status kvq_decode_step(const uint16_t *x_new, uint8_t *packed,
                            const int8_t *signs, kvq_rot rot, uint16_t *out,
                            kvq_stream stream);
 
+/*
+ * Decode step with a dequantized-prefix cache and an fp16 tail ("Quantization
+ * Speed Is Often a Kernel Problem", section "Before you celebrate...", second
+ * condition: the dequantized prefix is kept between steps instead of being
+ * recomputed, the last tokens stay in fp16, and the cache is refreshed when
+ * that window fills).  `kv` is the attention view the caller keeps across
+ * the steps of one sequence; a step touches O(window) rows, not O(pos).
+ *
+ * For every head h < n_heads:
+ *   - kv[h][pos] = x_new[h] exactly (fp16 tail);
+ *   - if (pos + 1) % window == 0, the window rows r in
+ *     [pos + 1 - window, pos] (kv rows, and x_new for r = pos) go through the
+ *     forward step into packed[h][r], scales[h][r], and kv[h][r] is replaced
+ *     by the inverse step of those codes.
+ * So after the call, kv rows of completed windows hold the dequantized
+ * values (identical to kvq_decode_step's output rows) and the rows of the
+ * open window hold the tokens themselves; packed/scales rows of the open
+ * window are not written.
+ *
+ *   x_new   [n_heads][d] fp16, 16-byte aligned (read)
+ *   packed  [n_heads][cap][d/2] uint8, 16-byte aligned (window rows written)
+ *   scales  [n_heads][cap][d/g] fp32, 4-byte aligned (window rows written)
+ *   kv      [n_heads][cap][d] fp16, 16-byte aligned (row pos written; on a
+ *           flush the window rows are read and rewritten)
+ *   n_heads >= 0 (0: no-op); cap >= 1; 0 <= pos < cap
+ *   window  1 <= window <= 4096 (16 in the pages' design)
+ *   other arguments as in kvq_rot_quant_fwd.
+ */
+kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *packed,
+                                    float *scales, uint16_t *kv,
+                                    int64_t n_heads, int64_t cap, int64_t pos,
+                                    int32_t window, int32_t d, int32_t group,
+                                    const int8_t *signs, kvq_rot rot,
+                                    kvq_stream stream);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *kvq_status_string(kvq_status s);
 

@@ -65,7 +65,7 @@ __all__ = [
     "sign_flip", "srft_matrix", "srht_matrix", "rotation_matrix",
     "rotate", "inverse_rotate", "quantize_groups", "dequantize_groups",
     "pack_nibbles", "unpack_nibbles", "rot_quant_fwd", "dequant_rot_inv",
-    "rotated_values", "near_tie_distance", "decode_step",
+    "rotated_values", "near_tie_distance", "decode_step", "decode_step_windowed",
 ]
 
 
@@ -269,3 +269,35 @@ def decode_step(x_new, packed_cache, scales_cache, pos: int, signs, rot: int,
     rows_s = scales_cache[:, : pos + 1, :].reshape(h * (pos + 1), d // group)
     out = dequant_rot_inv(rows_p, rows_s, signs, rot, group)
     return out.reshape(h, pos + 1, d)
+
+
+def decode_step_windowed(x_new, packed_cache, scales_cache, kv, pos: int, signs,
+                         rot: int, group: int, window: int = 16):
+    """Decode step with a dequantized-prefix cache and an fp16 tail.
+
+    [P1] "Before you celebrate...", second condition: the dequantized prefix
+    is cached between steps instead of recomputed, the last tokens (16 on
+    the pages) stay in fp16, and the cache is refreshed when that window
+    fills.  Reading: the window is the run of `window` positions ending at a
+    multiple of `window`; row pos of the view receives the new token as is;
+    when pos closes a window, the window's rows are quantized into the int4
+    cache and the view keeps their dequantized values.  Refreshing only the
+    closed window gives the same view as recomputing the whole prefix,
+    because rows of earlier windows keep their codes.
+
+    x_new: [H, d] fp16; packed_cache [H, cap, d/2] uint8, scales_cache
+    [H, cap, d/g] float32 and kv [H, cap, d] fp16 are updated in place.
+    """
+    x_new = np.asarray(x_new, dtype=np.float16)
+    h, d = x_new.shape
+    kv[:, pos, :] = x_new
+    if (pos + 1) % window != 0:
+        return kv
+    first = pos + 1 - window
+    rows = kv[:, first: pos + 1, :].reshape(h * window, d)
+    p_w, s_w = rot_quant_fwd(rows, signs, rot, group)
+    packed_cache[:, first: pos + 1, :] = p_w.reshape(h, window, d // 2)
+    scales_cache[:, first: pos + 1, :] = s_w.reshape(h, window, d // group)
+    kv[:, first: pos + 1, :] = dequant_rot_inv(p_w, s_w, signs, rot, group).reshape(
+        h, window, d)
+    return kv

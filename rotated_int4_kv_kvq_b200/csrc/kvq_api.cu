@@ -225,6 +225,32 @@ kvq_status kvq_decode_step(const uint16_t* x_new, uint8_t* packed, float* scales
   return from_cuda(e);
 }
 
+kvq_status kvq_decode_step_windowed(const uint16_t* x_new, uint8_t* packed, float* scales,
+                                    uint16_t* kv, int64_t n_heads, int64_t cap, int64_t pos,
+                                    int32_t window, int32_t d, int32_t group, const int8_t* signs,
+                                    kvq_rot rot, kvq_stream stream) {
+  if (kvq_status s = check_shape(d, group, rot)) return s;
+  if (n_heads < 0 || n_heads > kMaxRows || cap < 1 || cap > kMaxRows || pos < 0 || pos >= cap ||
+      window < 1 || window > 4096)
+    return KVQ_ERR_BAD_SIZE;
+  const int64_t ng = d / group;
+  if (n_heads * cap > kMaxRows || n_heads * cap * ng > kMaxRows ||
+      n_heads * int64_t(window) > kMaxRows)
+    return KVQ_ERR_BAD_SIZE;
+  if (!x_new || !packed || !scales || !kv || !signs) return KVQ_ERR_NULL;
+  if (!aligned(x_new, 16) || !aligned(packed, 16) || !aligned(scales, 4) || !aligned(kv, 16))
+    return KVQ_ERR_MISALIGNED;
+  if (n_heads == 0) return KVQ_OK;
+  DeviceInfo dev;
+  if (kvq_status s = device_info(&dev)) return s;
+  kvq::WindowLaunch W{x_new, packed, scales, kv, signs, n_heads, cap, pos, window, dev.sm_count,
+                      reinterpret_cast<cudaStream_t>(stream)};
+  cudaError_t e = d == 64    ? kvq::launch_window<64>(group, rot, W)
+                  : d == 128 ? kvq::launch_window<128>(group, rot, W)
+                             : kvq::launch_window<256>(group, rot, W);
+  return from_cuda(e);
+}
+
 const char* kvq_status_string(kvq_status s) {
   switch (s) {
     case KVQ_OK: return "ok";

@@ -55,7 +55,7 @@ struct Tuning {
   static constexpr int S_OUT = D == 64 ? 2 : KVQ_SOUT_BIG;
   static constexpr bool SRFT = ROT == kRotSRFT;
   static constexpr int FWD_MINB =
-      D == 64 ? KVQ_FWD_MINB_64 : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 3)
+      D == 64 ? (SRFT ? KVQ_FWD_MINB_64 : 4) : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 3)
                                         : (SRFT ? KVQ_FWD_MINB_256_SRFT : 3));
   static constexpr int INV_MINB =
       D == 64 ? KVQ_INV_MINB_64 : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 2)
@@ -175,32 +175,52 @@ cudaError_t decode_one(const DecodeLaunch& L) {
   return cudaGetLastError();
 }
 
+// Resident 256-thread blocks per SM of a one-warp-per-vector kernel (cached
+// per device).
+template <auto Kern>
+cudaError_t wide_occupancy(int* occ_out) {
+  static int occ[kMaxDevices];
+  static std::mutex mu;
+  int dev;
+  cudaError_t e = current_device(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  if (occ[dev] == 0) {
+    int b = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, Kern, kWideThreads, 0);
+    if (e != cudaSuccess) return e;
+    occ[dev] = std::max(b, 1);
+  }
+  *occ_out = occ[dev];
+  return cudaSuccess;
+}
+
+inline int wide_grid(int64_t rows, int sm_count, int occ) {
+  const int64_t want = (rows + kWideThreads / 32 - 1) / (kWideThreads / 32);
+  return int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count) * occ)));
+}
+
 template <int D, int G, int ROT>
 cudaError_t decode_wide_one(const DecodeWideLaunch& L) {
   constexpr auto kern = kvq_decode_wide_kernel<D, G, ROT>;
-  constexpr int threads = 256;
   int occ;
-  cudaError_t e;
-  {
-    static int occ_dev[kMaxDevices];
-    static std::mutex mu;
-    int dev;
-    e = current_device(&dev);
-    if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> g(mu);
-    if (occ_dev[dev] == 0) {
-      int b = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, threads, 0);
-      if (e != cudaSuccess) return e;
-      occ_dev[dev] = std::max(b, 1);
-    }
-    occ = occ_dev[dev];
-  }
+  cudaError_t e = wide_occupancy<kern>(&occ);
+  if (e != cudaSuccess) return e;
   DecodeWideArgs a{L.x_new, L.packed, L.scales, L.out, L.signs, L.n_heads, L.cap, L.pos};
-  const int64_t rows = L.n_heads * (L.pos + 1);
-  const int64_t want = (rows + threads / 32 - 1) / (threads / 32);
-  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(L.sm_count) * occ)));
-  kern<<<grid, threads, 0, L.stream>>>(a);
+  kern<<<wide_grid(L.n_heads * (L.pos + 1), L.sm_count, occ), kWideThreads, 0, L.stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int G, int ROT>
+cudaError_t window_one(const WindowLaunch& L) {
+  constexpr auto kern = kvq_window_wide_kernel<D, G, ROT>;
+  int occ;
+  cudaError_t e = wide_occupancy<kern>(&occ);
+  if (e != cudaSuccess) return e;
+  WindowArgs a{L.x_new, L.packed, L.scales, L.kv, L.signs, L.n_heads, L.cap, L.pos, L.window};
+  const bool flush = (L.pos + 1) % L.window == 0;
+  const int64_t rows = flush ? L.n_heads * L.window : L.n_heads;
+  kern<<<wide_grid(rows, L.sm_count, occ), kWideThreads, 0, L.stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -240,6 +260,10 @@ template <int D, int G, int ROT>
 struct DecodeWideOp {
   static cudaError_t run(const DecodeWideLaunch& l) { return decode_wide_one<D, G, ROT>(l); }
 };
+template <int D, int G, int ROT>
+struct WindowOp {
+  static cudaError_t run(const WindowLaunch& l) { return window_one<D, G, ROT>(l); }
+};
 
 }  // namespace detail
 
@@ -261,6 +285,11 @@ cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L) {
 template <int D>
 cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L) {
   return detail::dispatch<D, detail::DecodeWideOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t launch_window(int group, int rot, const WindowLaunch& L) {
+  return detail::dispatch<D, detail::WindowOp>(group, rot, L);
 }
 
 template <int D>

@@ -49,6 +49,18 @@ struct DecodeWideLaunch {
   cudaStream_t stream;
 };
 
+struct WindowLaunch {
+  const uint16_t* x_new;  // [n_heads][d]
+  uint8_t* packed;        // [n_heads][cap][d/2]
+  float* scales;          // [n_heads][cap][d/g]
+  uint16_t* kv;           // [n_heads][cap][d]
+  const int8_t* signs;
+  int64_t n_heads, cap, pos;
+  int window;
+  int sm_count;
+  cudaStream_t stream;
+};
+
 struct DecodeLaunch {
   const CUtensorMap* tmXn;  // x_new [n_heads][d], box {64, VPW}
   const CUtensorMap* tmQn;  // packed row pos of every head, box {d/2, VPW}
@@ -71,6 +83,8 @@ template <int D>
 cudaError_t launch_decode(int group, int rot, const DecodeLaunch& L);
 template <int D>
 cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L);
+template <int D>
+cudaError_t launch_window(int group, int rot, const WindowLaunch& L);
 // Reads (and optionally clears) the device status word of that translation
 // unit on the current device; the caller has synchronized the device.
 template <int D>

@@ -28,6 +28,7 @@
 namespace kvq {
 
 constexpr float kSqrt2Wide = 1.41421356237309504880f;
+constexpr int kWideThreads = 256;
 
 // exp(-2 pi i j / 256) for j < 256, rounded once from double.
 struct Tw256 {
@@ -286,26 +287,37 @@ struct DecodeWideArgs {
   int64_t n_heads, cap, pos;
 };
 
-template <int D, int ROT>
+// Loads through the read-only path unless RO is false (rows this kernel
+// also writes).
+template <bool RO, class T>
+__device__ __forceinline__ T wide_ld(const T* p) {
+  if constexpr (RO) {
+    return __ldg(p);
+  } else {
+    return *p;
+  }
+}
+
+template <int D, int ROT, bool RO = true>
 __device__ __forceinline__ void wide_load_words(const uint16_t* row, const WideLane<D, ROT>& L,
                                                 uint32_t (&xw)[Wide<D, ROT>::C]) {
   using P = Wide<D, ROT>;
   const uint32_t* w = reinterpret_cast<const uint32_t*>(row);
   if constexpr (ROT == kRotSRFT) {
 #pragma unroll
-    for (int j = 0; j < P::C; ++j) xw[j] = __ldg(w + L.lane + 32 * j) ^ L.mask[j];
+    for (int j = 0; j < P::C; ++j) xw[j] = wide_ld<RO>(w + L.lane + 32 * j) ^ L.mask[j];
   } else if constexpr (P::C == 4) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(w) + L.lane);
+    const uint4 v = wide_ld<RO>(reinterpret_cast<const uint4*>(w) + L.lane);
     xw[0] = v.x ^ L.mask[0];
     xw[1] = v.y ^ L.mask[1];
     xw[2] = v.z ^ L.mask[2];
     xw[3] = v.w ^ L.mask[3];
   } else if constexpr (P::C == 2) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(w) + L.lane);
+    const uint2 v = wide_ld<RO>(reinterpret_cast<const uint2*>(w) + L.lane);
     xw[0] = v.x ^ L.mask[0];
     xw[1] = v.y ^ L.mask[1];
   } else {
-    xw[0] = __ldg(w + L.lane) ^ L.mask[0];
+    xw[0] = wide_ld<RO>(w + L.lane) ^ L.mask[0];
   }
 }
 
@@ -342,79 +354,160 @@ __device__ __forceinline__ float wide_group_max(float m) {
   return m;
 }
 
-template <int D, int G, int ROT>
-__global__ void __launch_bounds__(256) kvq_decode_wide_kernel(const DecodeWideArgs a) {
+// Code bytes of the lane's chunk of one row.
+template <int D, int ROT>
+__device__ __forceinline__ void wide_store_code(uint8_t* qrow, const WideLane<D, ROT>& L,
+                                                uint32_t code) {
+  constexpr int QB = Wide<D, ROT>::W / 2;
+  if constexpr (QB == 4) {
+    reinterpret_cast<uint32_t*>(qrow)[L.k2] = code;
+  } else if constexpr (QB == 2) {
+    reinterpret_cast<uint16_t*>(qrow)[L.k2] = uint16_t(code);
+  } else {
+    qrow[L.k2] = uint8_t(code);
+  }
+}
+
+template <int D, int ROT>
+__device__ __forceinline__ uint32_t wide_load_code(const uint8_t* qrow, const WideLane<D, ROT>& L) {
+  constexpr int QB = Wide<D, ROT>::W / 2;
+  if constexpr (QB == 4) {
+    return __ldg(reinterpret_cast<const uint32_t*>(qrow) + L.k2);
+  } else if constexpr (QB == 2) {
+    return __ldg(reinterpret_cast<const uint16_t*>(qrow) + L.k2);
+  } else {
+    return __ldg(qrow + L.k2);
+  }
+}
+
+// Forward step on one fp16 row (steps a1-a5): writes the row's codes and
+// scales, returns this lane's code bytes and its group's scale.
+template <int D, int G, int ROT, bool RO = true>
+__device__ __forceinline__ void wide_quantize_row(const uint16_t* src, uint8_t* qrow, float* srow,
+                                                  const WideLane<D, ROT>& L, uint32_t& code,
+                                                  float& s) {
   using P = Wide<D, ROT>;
-  constexpr int NG = D / G;
   constexpr int GL = G / P::W;  // lanes (chunks) per group
-  constexpr int QB = P::W / 2;  // code bytes per lane
+  uint32_t xw[P::C];
+  wide_load_words<D, ROT, RO>(src, L, xw);
+  float Y[P::W];
+  wide_rotate_fwd<D, ROT>(xw, L, Y);
+  float m = fabsf(Y[0]);
+#pragma unroll
+  for (int j = 1; j < P::W; ++j) m = fmaxf(m, fabsf(Y[j]));
+  m = wide_group_max<D, G, ROT>(m);
+  const float inv = m > 0.0f ? __fdiv_rn(7.0f, m) : 0.0f;
+  s = m * P::KAPPA7;
+  uint32_t f[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    f[j] = j < P::W ? __float_as_uint(__fmaf_rn(Y[j], inv, kRoundMagic))
+                    : __float_as_uint(kRoundMagic);
+  code = pack8(f);
+  wide_store_code<D, ROT>(qrow, L, code);
+  if (L.k2 % GL == 0) srow[L.k2 / GL] = s;
+}
+
+// Inverse step on one row (steps a6-a7) from the lane's code bytes and
+// scale; writes the fp16 row.
+template <int D, int ROT>
+__device__ __forceinline__ void wide_dequant_row(uint32_t code, float s, uint16_t* dst,
+                                                 const WideLane<D, ROT>& L) {
+  using P = Wide<D, ROT>;
+  const f2 magic = mk2(kUnpackMagic, kUnpackMagic);
+  float Y[P::W];
+  {
+    f2 q[4];
+    unpack8(code, q);
+    const float sk = s * P::KAPPA;
+    const f2 sk2 = mk2(sk, sk);
+#pragma unroll
+    for (int j = 0; j < P::C; ++j) {
+      const f2 v = mul2(sub2(q[j], magic), sk2);
+      Y[2 * j] = lo2(v);
+      Y[2 * j + 1] = hi2(v);
+    }
+  }
+  uint32_t xo[P::C];
+  wide_rotate_inv<D, ROT>(Y, L, xo);
+  wide_store_words<D, ROT>(dst, L, xo);
+}
+
+template <int D, int G, int ROT>
+__global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const DecodeWideArgs a) {
+  constexpr int NG = D / G;
   const int lane = threadIdx.x & 31;
   WideLane<D, ROT> L;
   L.init(a.signs, lane);
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int64_t total = a.n_heads * (a.pos + 1);
-  const f2 magic = mk2(kUnpackMagic, kUnpackMagic);
   for (int64_t it = gw; it < total; it += nw) {
     const bool fresh = it < a.n_heads;
     const int64_t head = fresh ? it : (it - a.n_heads) / a.pos;
     const int64_t row = fresh ? a.pos : (it - a.n_heads) % a.pos;
     uint8_t* qrow = a.packed + (head * a.cap + row) * (D / 2);
     float* srow = a.scales + (head * a.cap + row) * NG;
-    uint32_t code;  // this lane's W codes (QB bytes)
+    uint32_t code;  // this lane's W codes
     float s;        // scale of this lane's group
     if (fresh) {
-      uint32_t xw[P::C];
-      wide_load_words<D, ROT>(a.x_new + head * D, L, xw);
-      float Y[P::W];
-      wide_rotate_fwd<D, ROT>(xw, L, Y);
-      float m = fabsf(Y[0]);
-#pragma unroll
-      for (int j = 1; j < P::W; ++j) m = fmaxf(m, fabsf(Y[j]));
-      m = wide_group_max<D, G, ROT>(m);
-      const float inv = m > 0.0f ? __fdiv_rn(7.0f, m) : 0.0f;
-      s = m * P::KAPPA7;
-      uint32_t f[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        f[j] = j < P::W ? __float_as_uint(__fmaf_rn(Y[j], inv, kRoundMagic))
-                        : __float_as_uint(kRoundMagic);
-      code = pack8(f);
-      if constexpr (QB == 4) {
-        reinterpret_cast<uint32_t*>(qrow)[L.k2] = code;
-      } else if constexpr (QB == 2) {
-        reinterpret_cast<uint16_t*>(qrow)[L.k2] = uint16_t(code);
-      } else {
-        qrow[L.k2] = uint8_t(code);
-      }
-      if (L.k2 % GL == 0) srow[L.k2 / GL] = s;
+      wide_quantize_row<D, G, ROT>(a.x_new + head * D, qrow, srow, L, code, s);
     } else {
-      if constexpr (QB == 4) {
-        code = __ldg(reinterpret_cast<const uint32_t*>(qrow) + L.k2);
-      } else if constexpr (QB == 2) {
-        code = __ldg(reinterpret_cast<const uint16_t*>(qrow) + L.k2);
-      } else {
-        code = __ldg(qrow + L.k2);
-      }
-      s = __ldg(srow + L.k2 / GL);
+      code = wide_load_code<D, ROT>(qrow, L);
+      s = __ldg(srow + L.k2 / (G / Wide<D, ROT>::W));
     }
-    // dequantize: Yin = q * s * KAPPA
-    float Y[P::W];
-    {
-      f2 q[4];
-      unpack8(code, q);
-      const float sk = s * P::KAPPA;
-      const f2 sk2 = mk2(sk, sk);
-#pragma unroll
-      for (int j = 0; j < P::C; ++j) {
-        const f2 v = mul2(sub2(q[j], magic), sk2);
-        Y[2 * j] = lo2(v);
-        Y[2 * j + 1] = hi2(v);
-      }
+    wide_dequant_row<D, ROT>(code, s, a.out + (head * (a.pos + 1) + row) * D, L);
+  }
+}
+
+// ------------------------------------------- windowed decode (prefix cache) ---
+
+struct WindowArgs {
+  const uint16_t* x_new;  // [n_heads][d]
+  uint8_t* packed;        // [n_heads][cap][d/2]
+  float* scales;          // [n_heads][cap][d/g]
+  uint16_t* kv;           // [n_heads][cap][d], persistent attention view
+  const int8_t* signs;
+  int64_t n_heads, cap, pos;
+  int window;
+};
+
+// Decode step with a dequantized-prefix cache and an fp16 tail ([P1]
+// "Before you celebrate...", second condition): row pos of kv receives the
+// new token exactly; when that completes a window of `window` rows, the
+// window's rows are quantized into the int4 cache and kv keeps their
+// dequantized values, so rows of completed windows read as dequantized and
+// the rest of the prefix is never recomputed.
+template <int D, int G, int ROT>
+__global__ void __launch_bounds__(kWideThreads) kvq_window_wide_kernel(const WindowArgs a) {
+  constexpr int NG = D / G;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const bool flush = (a.pos + 1) % a.window == 0;
+  if (!flush) {  // copy the new rows into the tail
+    for (int64_t h = gw; h < a.n_heads; h += nw) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x_new + h * D);
+      uint4* dst = reinterpret_cast<uint4*>(a.kv + (h * a.cap + a.pos) * D);
+      for (int c = lane; c < D / 8; c += 32) dst[c] = __ldg(src + c);
     }
-    uint32_t xo[P::C];
-    wide_rotate_inv<D, ROT>(Y, L, xo);
-    wide_store_words<D, ROT>(a.out + (head * (a.pos + 1) + row) * D, L, xo);
+    return;
+  }
+  WideLane<D, ROT> L;
+  L.init(a.signs, lane);
+  const int64_t first = a.pos + 1 - a.window;
+  const int64_t total = a.n_heads * a.window;
+  for (int64_t it = gw; it < total; it += nw) {
+    const int64_t head = it / a.window;
+    const int64_t row = first + it % a.window;
+    const uint16_t* src = row == a.pos ? a.x_new + head * D : a.kv + (head * a.cap + row) * D;
+    uint8_t* qrow = a.packed + (head * a.cap + row) * (D / 2);
+    float* srow = a.scales + (head * a.cap + row) * NG;
+    uint32_t code;
+    float s;
+    wide_quantize_row<D, G, ROT, false>(src, qrow, srow, L, code, s);
+    __syncwarp();  // every lane has read the source row before it is overwritten
+    wide_dequant_row<D, ROT>(code, s, a.kv + (head * a.cap + row) * D, L);
   }
 }
 

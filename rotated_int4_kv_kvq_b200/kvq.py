@@ -28,7 +28,8 @@ LIB_PATH = os.environ.get("KVQ_LIBRARY") or os.path.join(
     os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
 EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_decode_step",
-           "kvq_status_string", "kvq_device_status", "kvq_version")
+           "kvq_decode_step_windowed", "kvq_status_string", "kvq_device_status",
+           "kvq_version")
 
 
 class KVQError(RuntimeError):
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
     lib.kvq_dequant_rot_inv.restype = i32
     lib.kvq_decode_step.argtypes = [p, p, p, i64, i64, i64, i32, i32, p, i32, p, p]
     lib.kvq_decode_step.restype = i32
+    lib.kvq_decode_step_windowed.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, i32, p, i32, p]
+    lib.kvq_decode_step_windowed.restype = i32
     lib.kvq_status_string.argtypes = [i32]
     lib.kvq_status_string.restype = ctypes.c_char_p
     lib.kvq_device_status.argtypes = [i32]
@@ -147,6 +150,26 @@ def kvq_decode_step(x_new: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
                              _ptr(signs), rot, _ptr(out), _stream(stream))
     _raise("kvq_decode_step", st)
     return out
+
+
+def kvq_decode_step_windowed(x_new: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                             kv: torch.Tensor, pos: int, signs: torch.Tensor, rot: int, group: int,
+                             window: int = 16, stream=None):
+    """Decode step with a dequantized-prefix cache: kv [H, cap, d] fp16 is the
+    persistent attention view (row ``pos`` gets x_new; a completed window of
+    ``window`` rows is quantized into packed/scales and replaced by its
+    dequantized values).  Returns kv."""
+    h, d = x_new.shape
+    cap = packed.shape[1]
+    _check(x_new, "x_new", torch.float16, (h, d))
+    _check(packed, "packed", torch.uint8, (h, cap, d // 2))
+    _check(scales, "scales", torch.float32, (h, cap, d // group))
+    _check(kv, "kv", torch.float16, (h, cap, d))
+    _check(signs, "signs", torch.int8, (d,))
+    st = lib.kvq_decode_step_windowed(_ptr(x_new), _ptr(packed), _ptr(scales), _ptr(kv), h, cap,
+                                      pos, window, d, group, _ptr(signs), rot, _stream(stream))
+    _raise("kvq_decode_step_windowed", st)
+    return kv
 
 
 def kvq_device_status(clear: bool = True) -> int:

@@ -96,3 +96,21 @@ def test_empty_calls_are_noops(kvq):
     assert lib.kvq_rot_quant_fwd(A, 0, 64, 32, A, 0, A, A, None) == 0
     assert lib.kvq_dequant_rot_inv(A, A, 0, 256, 256, A, 1, A, None) == 0
     assert lib.kvq_decode_step(A, A, A, 0, 8, 3, 128, 64, A, 0, A, None) == 0
+
+
+def test_windowed_decode_host_checks(kvq):
+    lib = kvq.lib
+    win = lib.kvq_decode_step_windowed
+    # (x_new, packed, scales, kv, n_heads, cap, pos, window, d, group, signs, rot, stream)
+    assert win(A, A, A, A, 2, 8, 3, 16, 96, 32, A, 0, None) == 2
+    assert win(A, A, A, A, 2, 8, 3, 16, 64, 16, A, 0, None) == 3
+    assert win(A, A, A, A, 2, 8, 3, 16, 64, 32, A, 3, None) == 5
+    assert win(A, A, A, None, 2, 8, 3, 16, 64, 32, A, 0, None) == 1
+    assert win(None, A, A, A, 2, 8, 3, 16, 64, 32, A, 0, None) == 1
+    assert win(A, A, A, A + 8, 2, 8, 3, 16, 64, 32, A, 0, None) == 4
+    assert win(A, A, A + 2, A, 2, 8, 3, 16, 64, 32, A, 0, None) == 4
+    for window in (0, -3, 4097):
+        assert win(A, A, A, A, 2, 8, 3, window, 64, 32, A, 0, None) == 7
+    assert win(A, A, A, A, 2, 8, 8, 16, 64, 32, A, 0, None) == 7  # pos == cap
+    assert win(A, A, A, A, -1, 8, 3, 16, 64, 32, A, 0, None) == 7
+    assert win(A, A, A, A, 0, 8, 3, 16, 64, 32, A, 0, None) == 0  # no heads: no-op

@@ -223,6 +223,33 @@ def check_decode_step(rot=O.SRFT, d=64, group=32):
     assert np.array_equal(out, ref)
 
 
+def check_decode_windowed(rot=O.SRFT, d=64, group=32, window=4, steps=11):
+    """The windowed step against the plain decode step on the same tokens:
+    after every step the view's closed windows equal the plain step's
+    output rows and the open window holds the tokens themselves; a step
+    leaves rows before its window bit-identical; packed/scales rows of the
+    open window stay untouched."""
+    rng = np.random.default_rng(7)
+    H, cap = 2, steps + 3
+    signs = W.make_signs(d)
+    pc = np.zeros((H, cap, d // 2), np.uint8)
+    sc = np.zeros((H, cap, d // group), np.float32)
+    kv = np.zeros((H, cap, d), np.float16)
+    pc2 = np.zeros_like(pc)
+    sc2 = np.zeros_like(sc)
+    toks = (rng.standard_normal((steps, H, d)) * 3).astype(np.float16)
+    for pos in range(steps):
+        before = kv.copy()
+        O.decode_step_windowed(toks[pos], pc, sc, kv, pos, signs, rot, group, window)
+        out = O.decode_step(toks[pos], pc2, sc2, pos, signs, rot, group)
+        closed = ((pos + 1) // window) * window
+        assert np.array_equal(kv[:, :closed], out[:, :closed])
+        assert np.array_equal(kv[:, closed: pos + 1], toks[closed: pos + 1].transpose(1, 0, 2))
+        first = pos + 1 - window if (pos + 1) % window == 0 else pos
+        assert np.array_equal(kv[:, :first], before[:, :first])
+        assert not pc[:, closed:].any() and not sc[:, closed:].any()
+
+
 # ------------------------------------------------------------------ tests ---
 
 @pytest.mark.parametrize("d", [2, 4, 8, 64, 128, 256])
@@ -299,6 +326,12 @@ def test_zero_vectors_and_zero_groups(rot):
 
 def test_decode_step_is_fwd_then_inv():
     check_decode_step()
+
+
+@pytest.mark.parametrize("window", [1, 4, 16])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+def test_decode_windowed_matches_plain_decode(rot, window):
+    check_decode_windowed(rot, window=window, steps=2 * window + 3)
 
 
 def test_granularity_monotone():
@@ -402,6 +435,30 @@ def _mut_pack_swapped(q):
     return (nib[..., 1::2] | (nib[..., 0::2] << 4)).astype(np.uint8)
 
 
+def _mut_window_flush_early(x_new, packed_cache, scales_cache, kv, pos, signs, rot, group,
+                            window=16):
+    """Off by one: closes a window at pos % window == 0 instead of at its
+    last position."""
+    return _flush_if(pos > 0 and pos % window == 0, x_new, packed_cache, scales_cache, kv, pos,
+                     signs, rot, group, window)
+
+
+def _flush_if(cond, x_new, packed_cache, scales_cache, kv, pos, signs, rot, group, window):
+    x_new = np.asarray(x_new, dtype=np.float16)
+    h, d = x_new.shape
+    kv[:, pos, :] = x_new
+    if not cond:
+        return kv
+    first = max(0, pos + 1 - window)
+    n = pos + 1 - first
+    rows = kv[:, first: pos + 1, :].reshape(h * n, d)
+    p_w, s_w = O.rot_quant_fwd(rows, signs, rot, group)
+    packed_cache[:, first: pos + 1, :] = p_w.reshape(h, n, d // 2)
+    scales_cache[:, first: pos + 1, :] = s_w.reshape(h, n, d // group)
+    kv[:, first: pos + 1, :] = O.dequant_rot_inv(p_w, s_w, signs, rot, group).reshape(h, n, d)
+    return kv
+
+
 def _mut_inverse_no_transpose(y, rot):
     return np.asarray(y, np.float64) @ O.rotation_matrix(y.shape[-1], rot).T
 
@@ -427,6 +484,8 @@ MUTATIONS = [
      [check_pack_layout, lambda: check_worked_example("srht")]),
     ("inverse_rotate", _mut_inverse_no_transpose,
      [lambda: check_worked_example("srft")]),
+    ("decode_step_windowed", _mut_window_flush_early,
+     [lambda: check_decode_windowed(window=4)]),
 ]
 
 
