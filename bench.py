@@ -251,12 +251,14 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, warmup, sampler=None):
-    """Device time of `steps` fwd+inv passes; per-kernel sums via events."""
+def time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, warmup, sampler=None,
+                 lam=None):
+    """Device time of `steps` fwd+inv passes; per-kernel sums via events.
+    With `lam`, the per-channel lambda entry points."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
+        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream, lam=lam)
+        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream, lam=lam)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -265,9 +267,9 @@ def time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, warmup, samp
     start.record(stream)
     for k in range(steps):
         ev[k][0].record(stream)
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
+        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream, lam=lam)
         ev[k][1].record(stream)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
+        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream, lam=lam)
         ev[k][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -535,6 +537,17 @@ def run_suite(kvq, dev):
                         "us": us, "algo_gbs": algo / (us * 1e-6) / 1e9,
                         "fp16_gbs": n * d * 2 / (us * 1e-6) / 1e9,
                         "vec_per_s": n / (us * 1e-6), "frac": algo / (us * 1e-6) / 1e9 / peak})
+                if g == d:  # the per-channel lambda hook on the same workload
+                    lam = torch.exp(0.5 * torch.randn(d, generator=torch.Generator().manual_seed(d)))
+                    lam = lam.to(dev)
+                    tot, f, i = time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 3,
+                                             lam=lam)
+                    for name, ms in (("fwd", f), ("inv", i)):
+                        us = 1e3 * ms / steps
+                        res.setdefault("lambda", []).append({
+                            "d": d, "group": g, "rot": "srft" if rot == 0 else "srht",
+                            "dir": name, "us": us, "algo_gbs": algo / (us * 1e-6) / 1e9,
+                            "frac": algo / (us * 1e-6) / 1e9 / peak})
             del x, packed, scales, out
             torch.cuda.empty_cache()
     # decode: 26 layers x (K, V) x d=256, g=256; one call per layer (2 heads)

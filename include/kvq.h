@@ -117,6 +117,30 @@ kvq_status kvq_dequant_rot_inv(const uint8_t *packed, const float *scales,
                                kvq_stream stream);
 
 /*
+ * Forward and inverse steps with a per-channel factor lambda, the kernel
+ * hook of "Quantization Speed Is Often a Kernel Problem", section "Before you
+ * celebrate..." (first condition: per-channel lambda plus per-group
+ * abs-max, inside the fused kernel).  The pages do not define how lambda is
+ * calibrated, so it is an input:
+ *   forward: u = D (lambda * x) (channel-wise), then as kvq_rot_quant_fwd;
+ *   inverse: x_hat = (D R^T y_hat) / lambda (channel-wise, before the fp16
+ *            rounding), i.e. the inverse step of the same scaled space.
+ *   lambda  [d] fp32, 8-byte aligned DEVICE pointer (read); finite and
+ *           non-zero (not checked on the device).  NULL -> KVQ_ERR_NULL.
+ *   other arguments as in kvq_rot_quant_fwd / kvq_dequant_rot_inv.
+ */
+kvq_status kvq_rot_quant_fwd_lambda(const uint16_t *x, int64_t n_vec, int32_t d,
+                                    int32_t group, const int8_t *signs,
+                                    const float *lambda, kvq_rot rot,
+                                    uint8_t *packed, float *scales,
+                                    kvq_stream stream);
+kvq_status kvq_dequant_rot_inv_lambda(const uint8_t *packed, const float *scales,
+                                      int64_t n_vec, int32_t d, int32_t group,
+                                      const int8_t *signs, const float *lambda,
+                                      kvq_rot rot, uint16_t *out,
+                                      kvq_stream stream);
+
+/*
  * Decode step for one head-major cache, one launch ("A scene" and "First,
  * the 17%": every layer, every decoding step, the new K/V token is rotated
  * and quantized and the cache is dequantized for attention).

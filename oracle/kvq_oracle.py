@@ -202,33 +202,44 @@ def unpack_nibbles(packed) -> np.ndarray:
     return q
 
 
-def rotated_values(x_fp16, signs, rot: int) -> np.ndarray:
-    """y = R D x in float64 for fp16 rows x (exactly widened)."""
+def rotated_values(x_fp16, signs, rot: int, lam=None) -> np.ndarray:
+    """y = R D (lam * x) in float64 for fp16 rows x (exactly widened); lam is
+    an optional per-channel float32 factor (see rot_quant_fwd)."""
     x = np.asarray(x_fp16, dtype=np.float16).astype(np.float64)
+    if lam is not None:
+        x = x * np.asarray(lam, dtype=np.float32).astype(np.float64)
     return rotate(sign_flip(x, signs), rot)
 
 
-def rot_quant_fwd(x_fp16, signs, rot: int, group: int):
+def rot_quant_fwd(x_fp16, signs, rot: int, group: int, lam=None):
     """Forward step: sign flip -> rotation -> per-group absmax int4 -> pack.
 
     [P1] "First, the 17%" and "Fusing four steps...": the forward kernel does
     rotate plus quantize.  Returns (packed uint8 [n, d/2], scales f32 [n, d/g]).
+    With `lam`, every channel i is first multiplied by lam[i]: [P1] "Before
+    you celebrate...", first condition (per-channel lambda plus per-group
+    abs-max inside the fused kernel).  The pages leave lambda undefined; it is
+    an input here, applied before the sign flip and the rotation.
     """
-    y = rotated_values(x_fp16, signs, rot)
+    y = rotated_values(x_fp16, signs, rot, lam)
     q, s = quantize_groups(y, group)
     return pack_nibbles(q), s
 
 
-def dequant_rot_inv(packed, scales, signs, rot: int, group: int) -> np.ndarray:
+def dequant_rot_inv(packed, scales, signs, rot: int, group: int, lam=None) -> np.ndarray:
     """Inverse step: unpack -> y_hat = s q -> u = R^T y_hat -> x_hat = D u.
 
     [P1] "First, the 17%": dequantized and rotated back when attention reads
-    it.  The float64 result is rounded to float16 once (reading R8).
+    it.  The float64 result is rounded to float16 once (reading R8).  With
+    `lam`, channel i is divided by lam[i] before that rounding (the inverse of
+    rot_quant_fwd's scaling).
     """
     q = unpack_nibbles(packed)
     yh = dequantize_groups(q, scales, group)
-    u = inverse_rotate(yh, rot)
-    return sign_flip(u, signs).astype(np.float16)
+    u = sign_flip(inverse_rotate(yh, rot), signs)
+    if lam is not None:
+        u = u / np.asarray(lam, dtype=np.float32).astype(np.float64)
+    return u.astype(np.float16)
 
 
 def near_tie_distance(y, s, group: int) -> np.ndarray:

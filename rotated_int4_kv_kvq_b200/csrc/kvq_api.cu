@@ -121,17 +121,15 @@ kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR
 
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
 
-}  // namespace
-
-extern "C" {
-
-kvq_status kvq_rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
-                             const int8_t* signs, kvq_rot rot, uint8_t* packed, float* scales,
-                             kvq_stream stream) {
+kvq_status rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
+                         const int8_t* signs, const float* lambda, kvq_rot rot, uint8_t* packed,
+                         float* scales, kvq_stream stream) {
   if (kvq_status s = check_shape(d, group, rot)) return s;
   if (n_vec < 0 || n_vec > kMaxRows) return KVQ_ERR_BAD_SIZE;
   if (!x || !signs || !packed || !scales) return KVQ_ERR_NULL;
-  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 16)) return KVQ_ERR_MISALIGNED;
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 16) ||
+      (lambda && !aligned(lambda, 8)))
+    return KVQ_ERR_MISALIGNED;
   if (n_vec == 0) return KVQ_OK;
   DeviceInfo dev;
   if (kvq_status s = device_info(&dev)) return s;
@@ -139,7 +137,7 @@ kvq_status kvq_rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_
   if (!map_x(&tmX, x, d, uint64_t(n_vec), uint64_t(2 * d)) ||
       !map_q(&tmQ, packed, d, uint64_t(n_vec), uint64_t(d / 2)))
     return KVQ_ERR_CUDA;
-  kvq::FwdLaunch L{&tmX, &tmQ, signs, scales, n_vec, dev.sm_count,
+  kvq::FwdLaunch L{&tmX, &tmQ, signs, lambda, scales, n_vec, dev.sm_count,
                    reinterpret_cast<cudaStream_t>(stream)};
   cudaError_t e = d == 64    ? kvq::launch_fwd<64>(group, rot, L)
                   : d == 128 ? kvq::launch_fwd<128>(group, rot, L)
@@ -147,13 +145,15 @@ kvq_status kvq_rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_
   return from_cuda(e);
 }
 
-kvq_status kvq_dequant_rot_inv(const uint8_t* packed, const float* scales, int64_t n_vec,
-                               int32_t d, int32_t group, const int8_t* signs, kvq_rot rot,
-                               uint16_t* out, kvq_stream stream) {
+kvq_status dequant_rot_inv(const uint8_t* packed, const float* scales, int64_t n_vec, int32_t d,
+                           int32_t group, const int8_t* signs, const float* lambda, kvq_rot rot,
+                           uint16_t* out, kvq_stream stream) {
   if (kvq_status s = check_shape(d, group, rot)) return s;
   if (n_vec < 0 || n_vec > kMaxRows || n_vec * (d / group) > kMaxRows) return KVQ_ERR_BAD_SIZE;
   if (!packed || !scales || !signs || !out) return KVQ_ERR_NULL;
-  if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(out, 16)) return KVQ_ERR_MISALIGNED;
+  if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+      (lambda && !aligned(lambda, 8)))
+    return KVQ_ERR_MISALIGNED;
   if (n_vec == 0) return KVQ_OK;
   DeviceInfo dev;
   if (kvq_status s = device_info(&dev)) return s;
@@ -162,12 +162,43 @@ kvq_status kvq_dequant_rot_inv(const uint8_t* packed, const float* scales, int64
       !map_s(&tmS, scales, d, group, uint64_t(n_vec) * uint64_t(d / group)) ||
       !map_x(&tmX, out, d, uint64_t(n_vec), uint64_t(2 * d)))
     return KVQ_ERR_CUDA;
-  kvq::InvLaunch L{&tmQ, &tmS, &tmX, signs, n_vec, dev.sm_count,
+  kvq::InvLaunch L{&tmQ, &tmS, &tmX, signs, lambda, n_vec, dev.sm_count,
                    reinterpret_cast<cudaStream_t>(stream)};
   cudaError_t e = d == 64    ? kvq::launch_inv<64>(group, rot, L)
                   : d == 128 ? kvq::launch_inv<128>(group, rot, L)
                              : kvq::launch_inv<256>(group, rot, L);
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
+                             const int8_t* signs, kvq_rot rot, uint8_t* packed, float* scales,
+                             kvq_stream stream) {
+  return rot_quant_fwd(x, n_vec, d, group, signs, nullptr, rot, packed, scales, stream);
+}
+
+kvq_status kvq_dequant_rot_inv(const uint8_t* packed, const float* scales, int64_t n_vec,
+                               int32_t d, int32_t group, const int8_t* signs, kvq_rot rot,
+                               uint16_t* out, kvq_stream stream) {
+  return dequant_rot_inv(packed, scales, n_vec, d, group, signs, nullptr, rot, out, stream);
+}
+
+kvq_status kvq_rot_quant_fwd_lambda(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
+                                    const int8_t* signs, const float* lambda, kvq_rot rot,
+                                    uint8_t* packed, float* scales, kvq_stream stream) {
+  if (!lambda) return KVQ_ERR_NULL;
+  return rot_quant_fwd(x, n_vec, d, group, signs, lambda, rot, packed, scales, stream);
+}
+
+kvq_status kvq_dequant_rot_inv_lambda(const uint8_t* packed, const float* scales, int64_t n_vec,
+                                      int32_t d, int32_t group, const int8_t* signs,
+                                      const float* lambda, kvq_rot rot, uint16_t* out,
+                                      kvq_stream stream) {
+  if (!lambda) return KVQ_ERR_NULL;
+  return dequant_rot_inv(packed, scales, n_vec, d, group, signs, lambda, rot, out, stream);
 }
 
 kvq_status kvq_decode_step(const uint16_t* x_new, uint8_t* packed, float* scales,

@@ -304,13 +304,17 @@ __device__ __forceinline__ void pair_join_fwd(const f2 (&y)[C::D / 4], int t, f2
 // Y: this thread's E rotated coordinates as P pairs (local order of the
 // layout), unnormalized: the true y is KAPPA * Y.  Input: sign-flipped fp16
 // words.
-template <class C>
-__device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f2 (&Y)[C::P]) {
+// With LAM, the values are multiplied by the load-side lambda pairs at
+// `lam` (shared memory) first.
+template <class C, bool LAM = false>
+__device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f2 (&Y)[C::P],
+                                           uint32_t lam = 0) {
   if constexpr (C::ROT == kRotSRHT) {
 #pragma unroll
     for (int j = 0; j < C::NW; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
       Y[j] = mk2(f.x, f.y);
+      if constexpr (LAM) Y[j] = mul2(Y[j], lds_f2(lam + 8u * j));
     }
     fwht<C::P>(Y);
     if constexpr (C::TPV == 2) {  // H_d = [[H, H], [H, -H]] across the pair
@@ -327,6 +331,7 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
     for (int j = 0; j < C::NW; ++j) {
       const float2 f = half2_bits_to_float2(xw[j]);
       u[j] = mk2(f.x, f.y);
+      if constexpr (LAM) u[j] = mul2(u[j], lds_f2(lam + 8u * j));
     }
     RFFT2<C::E / 2>::fwd(u, y2);
     if constexpr (C::TPV == 1) {
@@ -411,8 +416,15 @@ __device__ __forceinline__ void pair_join_inv(const f2 (&Y)[C::P], int t, f2 (&Z
 // inverse of rotate_fwd's unnormalized map up to the factor 1/KAPPA^2) yields
 // u itself.  Words of a two-lane codelet output that carry polarity -1 are
 // corrected by the store-side sign mask.
-template <class C>
-__device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[C::NW]) {
+// With LAM, the values are multiplied by the store-side 1/lambda pairs at
+// `lam` (shared memory) before the fp16 rounding.
+template <class C, bool LAM = false>
+__device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[C::NW],
+                                           uint32_t lam = 0) {
+  auto scaled = [&](f2 v, int j) {
+    if constexpr (LAM) v = mul2(v, lds_f2(lam + 8u * j));
+    return float2_to_half2_bits(lo2(v), hi2(v));
+  };
   if constexpr (C::ROT == kRotSRHT) {
     if constexpr (C::TPV == 2) {
       const float sg = t ? -1.0f : 1.0f;
@@ -422,7 +434,7 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     }
     fwht<C::P>(Y);
 #pragma unroll
-    for (int j = 0; j < C::NW; ++j) xw[j] = float2_to_half2_bits(lo2(Y[j]), hi2(Y[j]));
+    for (int j = 0; j < C::NW; ++j) xw[j] = scaled(Y[j], j);
   } else {
     f2 z[C::NW], x2[C::NW];
     if constexpr (C::TPV == 1) {
@@ -435,7 +447,7 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     RFFT2<C::E / 2>::inv(z, x2);
     if constexpr (C::TPV == 1) {
 #pragma unroll
-      for (int n = 0; n < C::NW; ++n) xw[n] = float2_to_half2_bits(lo2(x2[n]), hi2(x2[n]));
+      for (int n = 0; n < C::NW; ++n) xw[n] = scaled(x2[n], n);
     } else {
       // Thread 0 holds the even samples e_m, thread 1 r_m = (-1)^m o_{m+NR/2}
       // (o: odd samples), as fp16 pairs P_i = (s_{2i}, s_{2i+1}).  Both keep
@@ -445,9 +457,8 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
       const uint32_t se = t ? 0x1054u : 0x5410u, so = t ? 0x3276u : 0x7632u;
 #pragma unroll
       for (int i = 0; i < C::NW / 2; ++i) {
-        const uint32_t own = float2_to_half2_bits(lo2(x2[i]), hi2(x2[i]));
-        const f2 v = x2[i + C::NW / 2];
-        const uint32_t r = __shfl_xor_sync(kFull, float2_to_half2_bits(lo2(v), hi2(v)), 1);
+        const uint32_t own = scaled(x2[i], i);
+        const uint32_t r = __shfl_xor_sync(kFull, scaled(x2[i + C::NW / 2], i + C::NW / 2), 1);
         xw[2 * i] = __byte_perm(own, r, se);
         xw[2 * i + 1] = __byte_perm(own, r, so);
       }
@@ -561,6 +572,7 @@ __device__ __forceinline__ void dequantize(const uint32_t (&qw)[C::NQ],
 
 struct FwdArgs {
   const int8_t* signs;
+  const float* lambda;  // per-channel factors (LAM kernels only)
   float* scales;
   int64_t n_vec;
   int64_t n_tiles;
@@ -568,6 +580,7 @@ struct FwdArgs {
 
 struct InvArgs {
   const int8_t* signs;
+  const float* lambda;  // per-channel factors (LAM kernels only)
   int64_t n_vec;
   int64_t n_tiles;
 };
@@ -582,6 +595,45 @@ struct DecodeArgs {
   int64_t tok_tiles;    // ceil(pos / VPW)
   int64_t n_tiles;      // n_new_tiles + n_heads * tok_tiles
 };
+
+// Per-channel factor (lambda) of the fp32 values a thread holds, as pairs in
+// the order of its words: load side (word j of load_x) and store side (the
+// pairs rotate_inv converts to fp16 itself).  Thread-pair SRFT: thread t's
+// load word j holds channels (4j + t, 4j + 2 + t); on the store side thread
+// 0 converts e_m = x_{2m} and thread 1 r_m = +-x_{2((m + NR/2) mod NR) + 1}.
+template <class C>
+__device__ __forceinline__ void lambda_channels(int t, int j, bool store, int& c0, int& c1) {
+  if constexpr (C::PAIR_RFFT) {
+    if (!store) {
+      c0 = 4 * j + t;
+      c1 = 4 * j + 2 + t;
+    } else if (t == 0) {
+      c0 = 4 * j;
+      c1 = 4 * j + 2;
+    } else {
+      constexpr int NR = C::E;
+      c0 = 2 * ((2 * j + NR / 2) % NR) + 1;
+      c1 = 2 * ((2 * j + 1 + NR / 2) % NR) + 1;
+    }
+  } else {
+    c0 = 2 * (t * C::NW + j);
+    c1 = c0 + 1;
+  }
+}
+
+// s_lam[0, d/2): lambda pairs of the load side, s_lam[d/2, d): 1/lambda
+// pairs of the store side, NW pairs per thread role t.
+template <class C>
+__device__ __forceinline__ void fill_lambda(const float* lambda, f2* s_lam) {
+  for (int i = threadIdx.x; i < C::D / 2; i += blockDim.x) {
+    const int t = i / C::NW, j = i % C::NW;
+    int c0, c1;
+    lambda_channels<C>(t, j, false, c0, c1);
+    s_lam[i] = mk2(lambda[c0], lambda[c1]);
+    lambda_channels<C>(t, j, true, c0, c1);
+    s_lam[C::D / 2 + i] = mk2(1.0f / lambda[c0], 1.0f / lambda[c1]);
+  }
+}
 
 // s_mask[0, d/2): load-side masks, s_mask[d/2, d): store-side masks, each
 // as NW words per thread role t.
@@ -653,7 +705,7 @@ __device__ __noinline__ void drain_and_fail(uint32_t bars, const Ring& r, unsign
   atomicOr(status, 1u);
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                    const FwdArgs a, unsigned* status) {
@@ -663,6 +715,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
   __shared__ __align__(16) uint32_t s_mask[C::D];
+  __shared__ __align__(16) f2 s_lam[LAM ? C::D : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = C::TPV == 2 ? (lane & 1) : 0;
@@ -673,6 +726,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t bars = smem_u32(&bars_sm[warp][0]);
 
   fill_sign_masks<C>(a.signs, s_mask);
+  if constexpr (LAM) fill_lambda<C>(a.lambda, s_lam);
   if (lane == 0) {
     for (int s = 0; s < S_IN; ++s) mbar_init(bars + 8u * s, 1);
     fence_mbar_init();
@@ -683,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
   __syncthreads();
   const uint32_t mask = smem_u32(s_mask) + uint32_t(t * C::NW * 4);
+  const uint32_t lam = smem_u32(s_lam) + uint32_t(t * C::NW * 8);
 
   const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
   const int64_t nw = int64_t(gridDim.x) * kWarps;
@@ -720,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
       }
     }
     f2 Y[C::P];
-    rotate_fwd<C>(xw, t, Y);
+    rotate_fwd<C, LAM>(xw, t, Y, lam);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
     quantize<C, G>(Y, qw, sc);
@@ -745,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_inv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmX, const InvArgs a, unsigned* status) {
@@ -757,6 +812,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
   __shared__ __align__(16) uint32_t s_mask[C::D];
+  __shared__ __align__(16) f2 s_lam[LAM ? C::D : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = C::TPV == 2 ? (lane & 1) : 0;
@@ -767,6 +823,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t bars = smem_u32(&bars_sm[warp][0]);
 
   fill_sign_masks<C>(a.signs, s_mask);
+  if constexpr (LAM) fill_lambda<C>(a.lambda, s_lam);
   if (lane == 0) {
     for (int s = 0; s < S_IN; ++s) mbar_init(bars + 8u * s, 1);
     fence_mbar_init();
@@ -778,6 +835,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
   __syncthreads();
   const uint32_t mask_st = smem_u32(s_mask) + uint32_t((C::D / 2 + t * C::NW) * 4);
+  const uint32_t lam_st = smem_u32(s_lam) + uint32_t((C::D / 2 + t * C::NW) * 8);
 
   const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
   const int64_t nw = int64_t(gridDim.x) * kWarps;
@@ -819,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     f2 Y[C::P];
     dequantize<C, G>(qw, sc, Y);
     uint32_t xw[C::NW];
-    rotate_inv<C>(Y, t, xw);
+    rotate_inv<C, LAM>(Y, t, xw, lam_st);
 
     const int o = int((ring.consumed - 1) % S_OUT);
     if (lane == 0) bulk_wait_read<S_OUT - 1>();

@@ -237,6 +237,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -276,6 +282,12 @@ __device__ __forceinline__ f2 mk2(float x, float y) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(x), "f"(y));
   return r;
 }
+// An f2 from shared memory (8-byte aligned address).
+__device__ __forceinline__ f2 lds_f2(uint32_t a) {
+  const uint2 v = lds64(a);
+  return mk2(__uint_as_float(v.x), __uint_as_float(v.y));
+}
+
 __device__ __forceinline__ float lo2(f2 a) {
   float x;
   asm("mov.b64 {%0, _}, %1;" : "=f"(x) : "l"(a.v));

@@ -117,10 +117,11 @@ inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
   return int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count) * occ)));
 }
 
-template <int D, int G, int ROT>
-cudaError_t fwd_one(const FwdLaunch& L) {
+template <int D, int G, int ROT, bool LAM>
+cudaError_t fwd_run(const FwdLaunch& L) {
   using T = Tuning<D, ROT>;
-  constexpr auto kern = kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, T::FWD_MINB>;
+  constexpr auto kern =
+      kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, T::FWD_MINB, LAM>;
   constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES, T::S_OUT>();
   int occ;
   unsigned* st;
@@ -128,15 +129,21 @@ cudaError_t fwd_one(const FwdLaunch& L) {
   if (e == cudaSuccess) e = status_ptr(&st);
   if (e != cudaSuccess) return e;
   constexpr int vpw = 32 / T::TPV;
-  FwdArgs a{L.signs, L.scales, L.n_vec, (L.n_vec + vpw - 1) / vpw};
+  FwdArgs a{L.signs, L.lambda, L.scales, L.n_vec, (L.n_vec + vpw - 1) / vpw};
   kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(*L.tmX, *L.tmQ, a, st);
   return cudaGetLastError();
 }
 
 template <int D, int G, int ROT>
-cudaError_t inv_one(const InvLaunch& L) {
+cudaError_t fwd_one(const FwdLaunch& L) {
+  return L.lambda ? fwd_run<D, G, ROT, true>(L) : fwd_run<D, G, ROT, false>(L);
+}
+
+template <int D, int G, int ROT, bool LAM>
+cudaError_t inv_run(const InvLaunch& L) {
   using T = Tuning<D, ROT>;
-  constexpr auto kern = kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB>;
+  constexpr auto kern =
+      kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB, LAM>;
   constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT>();
   int occ;
   unsigned* st;
@@ -144,10 +151,15 @@ cudaError_t inv_one(const InvLaunch& L) {
   if (e == cudaSuccess) e = status_ptr(&st);
   if (e != cudaSuccess) return e;
   constexpr int vpw = 32 / T::TPV;
-  InvArgs a{L.signs, L.n_vec, (L.n_vec + vpw - 1) / vpw};
+  InvArgs a{L.signs, L.lambda, L.n_vec, (L.n_vec + vpw - 1) / vpw};
   kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(*L.tmQ, *L.tmS,
                                                                              *L.tmX, a, st);
   return cudaGetLastError();
+}
+
+template <int D, int G, int ROT>
+cudaError_t inv_one(const InvLaunch& L) {
+  return L.lambda ? inv_run<D, G, ROT, true>(L) : inv_run<D, G, ROT, false>(L);
 }
 
 template <int D, int G, int ROT>

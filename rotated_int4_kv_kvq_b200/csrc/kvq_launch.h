@@ -18,6 +18,7 @@ struct FwdLaunch {
   const CUtensorMap* tmX;  // x      [n_vec][d] fp16, box {64, VPW}, swizzle 128B
   const CUtensorMap* tmQ;  // packed [n_vec][d/2] u8, box {d/2, VPW}, swizzle = pitch
   const int8_t* signs;
+  const float* lambda;     // per-channel factors [d] or NULL
   float* scales;
   int64_t n_vec;
   int sm_count;
@@ -29,6 +30,7 @@ struct InvLaunch {
   const CUtensorMap* tmS;  // scales as 1-D f32, box {VPW * d/g}
   const CUtensorMap* tmX;  // out, as x above
   const int8_t* signs;
+  const float* lambda;     // per-channel factors [d] or NULL
   int64_t n_vec;
   int sm_count;
   cudaStream_t stream;

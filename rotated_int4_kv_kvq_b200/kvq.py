@@ -27,9 +27,9 @@ STATUS = {
 LIB_PATH = os.environ.get("KVQ_LIBRARY") or os.path.join(
     os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
-EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_decode_step",
-           "kvq_decode_step_windowed", "kvq_status_string", "kvq_device_status",
-           "kvq_version")
+EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_rot_quant_fwd_lambda",
+           "kvq_dequant_rot_inv_lambda", "kvq_decode_step", "kvq_decode_step_windowed",
+           "kvq_status_string", "kvq_device_status", "kvq_version")
 
 
 class KVQError(RuntimeError):
@@ -49,6 +49,10 @@ def _load() -> ctypes.CDLL:
     lib.kvq_rot_quant_fwd.restype = i32
     lib.kvq_dequant_rot_inv.argtypes = [p, p, i64, i32, i32, p, i32, p, p]
     lib.kvq_dequant_rot_inv.restype = i32
+    lib.kvq_rot_quant_fwd_lambda.argtypes = [p, i64, i32, i32, p, p, i32, p, p, p]
+    lib.kvq_rot_quant_fwd_lambda.restype = i32
+    lib.kvq_dequant_rot_inv_lambda.argtypes = [p, p, i64, i32, i32, p, p, i32, p, p]
+    lib.kvq_dequant_rot_inv_lambda.restype = i32
     lib.kvq_decode_step.argtypes = [p, p, p, i64, i64, i64, i32, i32, p, i32, p, p]
     lib.kvq_decode_step.restype = i32
     lib.kvq_decode_step_windowed.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, i32, p, i32, p]
@@ -97,9 +101,12 @@ def _raise(fn: str, st: int):
 
 def kvq_rot_quant_fwd(x: torch.Tensor, signs: torch.Tensor, rot: int, group: int,
                       packed: torch.Tensor | None = None,
-                      scales: torch.Tensor | None = None, stream=None):
+                      scales: torch.Tensor | None = None, stream=None,
+                      lam: torch.Tensor | None = None):
     """Forward step on x [n_vec, d] fp16 -> (packed [n_vec, d/2] u8,
-    scales [n_vec, d/group] f32).  Outputs are allocated when not given."""
+    scales [n_vec, d/group] f32).  Outputs are allocated when not given.
+    With ``lam`` ([d] f32), x is scaled channel-wise first
+    (kvq_rot_quant_fwd_lambda)."""
     n, d = x.shape
     _check(x, "x", torch.float16, (n, d))
     _check(signs, "signs", torch.int8, (d,))
@@ -109,15 +116,24 @@ def kvq_rot_quant_fwd(x: torch.Tensor, signs: torch.Tensor, rot: int, group: int
         scales = torch.empty((n, d // group), dtype=torch.float32, device=x.device)
     _check(packed, "packed", torch.uint8, (n, d // 2))
     _check(scales, "scales", torch.float32, (n, d // group))
-    st = lib.kvq_rot_quant_fwd(_ptr(x), n, d, group, _ptr(signs), rot, _ptr(packed),
-                               _ptr(scales), _stream(stream))
-    _raise("kvq_rot_quant_fwd", st)
+    if lam is None:
+        st = lib.kvq_rot_quant_fwd(_ptr(x), n, d, group, _ptr(signs), rot, _ptr(packed),
+                                   _ptr(scales), _stream(stream))
+        _raise("kvq_rot_quant_fwd", st)
+    else:
+        _check(lam, "lam", torch.float32, (d,))
+        st = lib.kvq_rot_quant_fwd_lambda(_ptr(x), n, d, group, _ptr(signs), _ptr(lam), rot,
+                                          _ptr(packed), _ptr(scales), _stream(stream))
+        _raise("kvq_rot_quant_fwd_lambda", st)
     return packed, scales
 
 
 def kvq_dequant_rot_inv(packed: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor,
-                        rot: int, group: int, out: torch.Tensor | None = None, stream=None):
-    """Inverse step -> out [n_vec, d] fp16 (allocated when not given)."""
+                        rot: int, group: int, out: torch.Tensor | None = None, stream=None,
+                        lam: torch.Tensor | None = None):
+    """Inverse step -> out [n_vec, d] fp16 (allocated when not given).  With
+    ``lam`` ([d] f32) the result is divided channel-wise by it
+    (kvq_dequant_rot_inv_lambda)."""
     n, half = packed.shape
     d = 2 * half
     _check(packed, "packed", torch.uint8, (n, half))
@@ -126,9 +142,16 @@ def kvq_dequant_rot_inv(packed: torch.Tensor, scales: torch.Tensor, signs: torch
     if out is None:
         out = torch.empty((n, d), dtype=torch.float16, device=packed.device)
     _check(out, "out", torch.float16, (n, d))
-    st = lib.kvq_dequant_rot_inv(_ptr(packed), _ptr(scales), n, d, group, _ptr(signs), rot,
-                                 _ptr(out), _stream(stream))
-    _raise("kvq_dequant_rot_inv", st)
+    if lam is None:
+        st = lib.kvq_dequant_rot_inv(_ptr(packed), _ptr(scales), n, d, group, _ptr(signs), rot,
+                                     _ptr(out), _stream(stream))
+        _raise("kvq_dequant_rot_inv", st)
+    else:
+        _check(lam, "lam", torch.float32, (d,))
+        st = lib.kvq_dequant_rot_inv_lambda(_ptr(packed), _ptr(scales), n, d, group,
+                                            _ptr(signs), _ptr(lam), rot, _ptr(out),
+                                            _stream(stream))
+        _raise("kvq_dequant_rot_inv_lambda", st)
     return out
 
 

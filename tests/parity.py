@@ -44,13 +44,15 @@ def _sat(v):
     return np.where(np.isinf(v), np.sign(v) * 65536.0, v)
 
 
-def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP_FRACTION):
+def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP_FRACTION,
+              lam=None):
     """Return (codes, scales, flips, max scale rel err, flipped-row mask).
 
     `max_flip_fraction` bounds near-tie flips on realistic data; structured
-    inputs (e.g. +-c vectors, whose rotations hit exact ties) pass None."""
+    inputs (e.g. +-c vectors, whose rotations hit exact ties) pass None.
+    `lam`: per-channel factor of the lambda entry points."""
     x16 = np.asarray(x16, dtype=np.float16)
-    y = O.rotated_values(x16, signs, rot)
+    y = O.rotated_values(x16, signs, rot, lam)
     q_ref, s_ref = O.quantize_groups(y, group)
     s = np.asarray(scales, dtype=np.float32)
     q = O.unpack_nibbles(np.asarray(packed, dtype=np.uint8))
@@ -78,21 +80,27 @@ def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP
     return q, s, flips, max_rel, bad.any(axis=1)
 
 
-def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None):
+def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None, lam=None):
     """x_hat of the GPU against the oracle inverse of the same codes/scales,
-    and against the oracle's own x_hat on rows without a code flip."""
+    and against the oracle's own x_hat on rows without a code flip.  With
+    `lam` the tolerance follows the channel scaling: the error of lam * x_hat
+    is bounded like that of an unscaled x_hat."""
     x = np.asarray(x16, dtype=np.float16).astype(np.float64)
     tol = XHAT_ATOL_REL * np.maximum(np.abs(x).max(axis=1, keepdims=True), 1e-30)
+    if lam is not None:
+        lam64 = np.asarray(lam, np.float32).astype(np.float64)
+        tol = XHAT_ATOL_REL * np.maximum(np.abs(x * lam64).max(axis=1, keepdims=True),
+                                         1e-30) / lam64 + np.float64(2.0 ** -24)
     with np.errstate(over="ignore"):
-        ref = _sat(O.dequant_rot_inv(packed, scales, signs, rot, group))
+        ref = _sat(O.dequant_rot_inv(packed, scales, signs, rot, group, lam))
     got = _sat(np.asarray(out, dtype=np.float16))
     err = np.abs(got - ref)
     inv_err = float((err / tol).max(initial=0.0))
     assert np.all(err <= tol), f"inverse error {inv_err:.3g} x tolerance"
     e2e = 0.0
-    p_ref, s_ref = O.rot_quant_fwd(np.asarray(x16, np.float16), signs, rot, group)
+    p_ref, s_ref = O.rot_quant_fwd(np.asarray(x16, np.float16), signs, rot, group, lam)
     with np.errstate(over="ignore"):
-        full = _sat(O.dequant_rot_inv(p_ref, s_ref, signs, rot, group))
+        full = _sat(O.dequant_rot_inv(p_ref, s_ref, signs, rot, group, lam))
     rows = np.ones(x.shape[0], bool) if flipped_rows is None else ~flipped_rows
     if rows.any():
         e = np.abs(got[rows] - full[rows]) / tol[rows]

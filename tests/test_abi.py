@@ -114,3 +114,17 @@ def test_windowed_decode_host_checks(kvq):
     assert win(A, A, A, A, 2, 8, 8, 16, 64, 32, A, 0, None) == 7  # pos == cap
     assert win(A, A, A, A, -1, 8, 3, 16, 64, 32, A, 0, None) == 7
     assert win(A, A, A, A, 0, 8, 3, 16, 64, 32, A, 0, None) == 0  # no heads: no-op
+
+
+def test_lambda_host_checks(kvq):
+    lib = kvq.lib
+    fwd, inv = lib.kvq_rot_quant_fwd_lambda, lib.kvq_dequant_rot_inv_lambda
+    # (x, n, d, g, signs, lambda, rot, packed, scales, stream)
+    assert fwd(A, 10, 64, 32, A, None, 0, A, A, None) == 1
+    assert inv(A, A, 10, 64, 32, A, None, 0, A, None) == 1
+    assert fwd(A, 10, 64, 32, A, A + 4, 0, A, A, None) == 4
+    assert inv(A, A, 10, 64, 32, A, A + 4, 0, A, None) == 4
+    assert fwd(A, 10, 96, 32, A, A, 0, A, A, None) == 2
+    assert inv(A, A, 10, 64, 16, A, A, 0, A, None) == 3
+    assert fwd(A, 0, 64, 32, A, A, 0, A, A, None) == 0
+    assert inv(A, A, 0, 64, 32, A, A, 1, A, None) == 0

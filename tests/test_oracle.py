@@ -250,6 +250,32 @@ def check_decode_windowed(rot=O.SRFT, d=64, group=32, window=4, steps=11):
         assert not pc[:, closed:].any() and not sc[:, closed:].any()
 
 
+def check_lambda(rot=O.SRFT, d=64, group=32):
+    """The per-channel lambda hook against the plain steps: lambda = 1 is the
+    plain step; a constant power of two scales only the scales; per-channel
+    powers of two equal the plain step on the pre-scaled fp16 input (exact),
+    and the inverse divides channel-wise."""
+    rng = np.random.default_rng(11)
+    signs = W.make_signs(d)
+    x = (rng.standard_normal((9, d)) * 3).astype(np.float16)
+    p0, s0 = O.rot_quant_fwd(x, signs, rot, group)
+    p1, s1 = O.rot_quant_fwd(x, signs, rot, group, np.ones(d, np.float32))
+    assert np.array_equal(p0, p1) and np.array_equal(s0, s1)
+    p4, s4 = O.rot_quant_fwd(x, signs, rot, group, np.full(d, 4.0, np.float32))
+    assert np.array_equal(p4, p0) and np.array_equal(s4, (4 * s0).astype(np.float32))
+    assert np.array_equal(O.dequant_rot_inv(p4, s4, signs, rot, group, np.full(d, 4.0, np.float32)),
+                          O.dequant_rot_inv(p0, s0, signs, rot, group))
+    lam = (2.0 ** rng.integers(-1, 3, d)).astype(np.float32)
+    xs = (x.astype(np.float64) * lam).astype(np.float16)
+    assert np.array_equal(xs.astype(np.float64), x.astype(np.float64) * lam)  # exact
+    pl, sl = O.rot_quant_fwd(x, signs, rot, group, lam)
+    pr, sr = O.rot_quant_fwd(xs, signs, rot, group)
+    assert np.array_equal(pl, pr) and np.array_equal(sl, sr)
+    xi = O.dequant_rot_inv(pl, sl, signs, rot, group, lam).astype(np.float64)
+    xr = O.dequant_rot_inv(pr, sr, signs, rot, group).astype(np.float64)
+    assert np.array_equal(xi, xr / lam)
+
+
 # ------------------------------------------------------------------ tests ---
 
 @pytest.mark.parametrize("d", [2, 4, 8, 64, 128, 256])
@@ -332,6 +358,12 @@ def test_decode_step_is_fwd_then_inv():
 @pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
 def test_decode_windowed_matches_plain_decode(rot, window):
     check_decode_windowed(rot, window=window, steps=2 * window + 3)
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("d,group", [(64, 32), (256, 256)])
+def test_lambda_hook(rot, d, group):
+    check_lambda(rot, d, group)
 
 
 def test_granularity_monotone():
@@ -459,6 +491,15 @@ def _flush_if(cond, x_new, packed_cache, scales_cache, kv, pos, signs, rot, grou
     return kv
 
 
+def _mut_lambda_after_rotation(x_fp16, signs, rot, lam=None):
+    # lambda applied to y instead of x
+    x = np.asarray(x_fp16, dtype=np.float16).astype(np.float64)
+    y = O.rotate(O.sign_flip(x, signs), rot)
+    if lam is not None:
+        y = y * np.asarray(lam, np.float32).astype(np.float64)
+    return y
+
+
 def _mut_inverse_no_transpose(y, rot):
     return np.asarray(y, np.float64) @ O.rotation_matrix(y.shape[-1], rot).T
 
@@ -486,6 +527,7 @@ MUTATIONS = [
      [lambda: check_worked_example("srft")]),
     ("decode_step_windowed", _mut_window_flush_early,
      [lambda: check_decode_windowed(window=4)]),
+    ("rotated_values", _mut_lambda_after_rotation, [check_lambda]),
 ]
 
 
