@@ -349,6 +349,11 @@ def main():
     ap.add_argument("--group", type=int, default=64)
     ap.add_argument("--n-vec", type=int, default=1 << 21)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--attn-len", type=int, default=0,
+                    help="with --profile: decode attention over this many cached rows "
+                         "(--d, --group, --rot; --attn-heads KV heads, --attn-nq queries)")
+    ap.add_argument("--attn-heads", type=int, default=32)
+    ap.add_argument("--attn-nq", type=int, default=1)
     ap.add_argument("--decode-pos", type=int, default=0,
                     help="with --profile: run --reps 26-layer decode steps at this position")
     args = ap.parse_args()
@@ -465,6 +470,8 @@ def run_profile_case(args):
     dev = torch.device("cuda", 0)
     if args.decode_pos > 0:
         return run_profile_decode(kvq, dev, args)
+    if args.attn_len > 0:
+        return run_profile_attn(kvq, dev, args)
     d, g = args.d, args.group
     tokens = 8192
     heads = max(1, -(-args.n_vec // (2 * tokens)))
@@ -481,6 +488,27 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": {"d": d, "group": g, "rot": args.rot,
                                        "n_vec": int(x.shape[0]), "reps": args.reps,
                                        "status": st}}))
+    if st != 0:
+        sys.exit(1)
+
+
+def run_profile_attn(kvq, dev, args):
+    """`reps` decode-attention calls over `attn_len` cached rows."""
+    d, g, h, nq, n = args.d, args.group, args.attn_heads, args.attn_nq, args.attn_len
+    gen = torch.Generator(device=dev).manual_seed(5)
+    signs = torch.from_numpy(W.make_signs(d)).to(dev)
+    c = []
+    for _ in range(2):
+        x = torch.randn((h * n, d), generator=gen, device=dev).half()
+        p, s = kvq.kvq_rot_quant_fwd(x, signs, args.rot, g)
+        c += [p.reshape(h, n, -1), s.reshape(h, n, -1)]
+    q = torch.randn((h, nq, d), generator=gen, device=dev).half()
+    for _ in range(args.reps):
+        o = kvq.kvq_attend_decode(q, c[0], c[1], c[2], c[3], n, signs, args.rot, g)
+    torch.cuda.synchronize()
+    st = kvq.kvq_device_status()
+    print(json.dumps({"profile_attn": {"d": d, "group": g, "heads": h, "nq": nq, "len": n,
+                                       "status": st, "out0": float(o[0, 0, 0])}}))
     if st != 0:
         sys.exit(1)
 
@@ -612,7 +640,72 @@ def run_suite(kvq, dev):
                                   "algo_bytes_per_step": byts,
                                   "ideal_us": byts / (peak * 1e9) * 1e6})
     res["decode_windowed"] = run_window_suite(kvq, dev, seq, signs, peak)
+    res["attention"] = run_attention_suite(kvq, dev, peak)
     return res
+
+
+def graph_time_us(fn, reps=20):
+    """Per-call device time of fn() replayed as a CUDA graph."""
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    s2 = torch.cuda.Stream()
+    s2.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s2):
+        fn()
+    torch.cuda.current_stream().wait_stream(s2)
+    with torch.cuda.graph(gr):
+        fn()
+    for _ in range(2):
+        gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del gr
+    return 1e3 * e0.elapsed_time(e1) / reps
+
+
+def run_attention_suite(kvq, dev, peak):
+    """Decode attention reading the int4 cache: the Gemma-3-1B step (26
+    layers, 1 KV head with 4 queries, d = g = 256) as a graph of 26 calls, and
+    one SmolLM2-1.7B-shaped layer (32 KV heads, 1 query each, d = g = 64) for
+    throughput against the HBM roofline (codes + scales of K and V)."""
+    out = []
+    gen = torch.Generator(device=dev).manual_seed(21)
+    cases = [("gemma-3-1b step", 26, 1, 4, 256, 256, (256, 1024, 2048, 4096)),
+             ("smollm2-1.7b layer", 1, 32, 1, 64, 64, (1024, 4096, 16384))]
+    for name, layers, heads, nq, d, g, lens in cases:
+        cap = max(lens)
+        signs = torch.from_numpy(W.make_signs(d)).to(dev)
+        for rot in (kvq.SRFT, kvq.SRHT):
+            caches = []
+            for _ in range(layers):
+                c = []
+                for _kv in range(2):
+                    x = (torch.randn((heads * cap, d), generator=gen, device=dev)).half()
+                    p, s = kvq.kvq_rot_quant_fwd(x, signs, rot, g)
+                    c += [p.reshape(heads, cap, -1), s.reshape(heads, cap, -1)]
+                q = torch.randn((heads, nq, d), generator=gen, device=dev).half()
+                o = torch.empty((heads, nq, d), dtype=torch.float16, device=dev)
+                caches.append((q, c, o))
+            for n in lens:
+                def fn():
+                    for q, (kp, ks, vp, vs), o in caches:
+                        kvq.kvq_attend_decode(q, kp, ks, vp, vs, n, signs, rot, g, out=o)
+                us = graph_time_us(fn)
+                byts = layers * heads * n * 2 * fwd_bytes(d, g) - layers * heads * n * 2 * 2 * d
+                out.append({"workload": name, "rot": "srft" if rot == 0 else "srht",
+                            "len": n, "graph_us": us, "calls": layers,
+                            "algo_bytes": byts, "algo_gbs": byts / (us * 1e-6) / 1e9,
+                            "frac": byts / (us * 1e-6) / 1e9 / peak})
+            del caches
+            torch.cuda.empty_cache()
+    return out
 
 
 def run_window_suite(kvq, dev, seq, signs, peak, window=16):

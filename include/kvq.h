@@ -201,6 +201,39 @@ kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *packed,
                                     const int8_t *signs, kvq_rot rot,
                                     kvq_stream stream);
 
+/*
+ * Decode attention that reads the int4 cache directly ("Day 9 -
+ * Quantization: Shrink the Bytes Themselves", section "Decode into HBM, or
+ * Decode into Registers": the dequantization happens inside the consuming
+ * kernel; "Quantization Speed Is Often a Kernel Problem", "First, the 17%":
+ * K and V are dequantized and rotated back when attention reads them).
+ *
+ * For every KV head h < n_kv_heads and query i < n_q, with
+ * K_t = D R^T (s q)_K[h][t] and V_t likewise for t < len (exact, not
+ * rounded to fp16):
+ *   s_t = sm_scale <q[h][i], K_t>,  p = softmax(s),
+ *   out[h][i] = sum_t p_t V_t, rounded to fp16.
+ * Only codes and scales are read from memory: the kernel rotates each query
+ * once (R orthonormal: <q, D R^T y> = <R D q, y>), accumulates
+ * sum_t p_t y_V,t in the rotated domain and rotates back once per query.
+ *
+ *   q         [n_kv_heads][n_q][d] fp16, 16-byte aligned (read)
+ *   k_packed, v_packed  [n_kv_heads][cap][d/2] uint8, 16-byte aligned (read)
+ *   k_scales, v_scales  [n_kv_heads][cap][d/g] fp32, 4-byte aligned (read)
+ *   n_kv_heads 0..65535 (0: no-op); n_q 1..8 queries per KV head (GQA)
+ *   cap >= 1; 1 <= len <= cap (rows [0, len) are attended)
+ *   sm_scale  finite softmax scale (e.g. 1/sqrt(d))
+ *   out       [n_kv_heads][n_q][d] fp16, 16-byte aligned (written)
+ *   signs, rot, d, group as in kvq_rot_quant_fwd (the D and R the cache
+ *   was written with).
+ */
+kvq_status kvq_attend_decode(const uint16_t *q, const uint8_t *k_packed,
+                             const float *k_scales, const uint8_t *v_packed,
+                             const float *v_scales, int64_t n_kv_heads,
+                             int32_t n_q, int64_t cap, int64_t len, int32_t d,
+                             int32_t group, const int8_t *signs, kvq_rot rot,
+                             float sm_scale, uint16_t *out, kvq_stream stream);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *kvq_status_string(kvq_status s);
 

@@ -19,6 +19,10 @@ transforms.  Every function cites the passage it follows.  Sources:
 * [P4] "Quantization & Serving" (gowda.ai/ml-refresh/quantization.html):
   symmetric absmax quantization, x_hat_i = s q_i, rounding error at most s/2
   before clipping.
+* [P3] "Day 9 - Quantization: Shrink the Bytes Themselves"
+  (guan404ming.com/blog/9), section "Decode into HBM, or Decode into
+  Registers": the dequantization belongs inside the consuming kernel, so the
+  decoded values live only in registers.
 * [P5] "Chapter 25 - Quantization: The Hardware View"
   (karam-nus.github.io/chips/25_quantization_hardware_view.html), section
   "Kernels: Marlin, CUTLASS, and Why INT4 Packing Needs Special Code": two
@@ -66,6 +70,7 @@ __all__ = [
     "rotate", "inverse_rotate", "quantize_groups", "dequantize_groups",
     "pack_nibbles", "unpack_nibbles", "rot_quant_fwd", "dequant_rot_inv",
     "rotated_values", "near_tie_distance", "decode_step", "decode_step_windowed",
+    "dequant_rotated_f64", "attend_decode",
 ]
 
 
@@ -312,3 +317,40 @@ def decode_step_windowed(x_new, packed_cache, scales_cache, kv, pos: int, signs,
     kv[:, first: pos + 1, :] = dequant_rot_inv(p_w, s_w, signs, rot, group).reshape(
         h, window, d)
     return kv
+
+
+def dequant_rotated_f64(packed, scales, signs, rot: int, group: int) -> np.ndarray:
+    """x_hat = D R^T y_hat in float64, without dequant_rot_inv's final fp16
+    rounding: the value attention consumes when the dequantization happens
+    inside it ([P3] "Decode into HBM, or Decode into Registers")."""
+    q = unpack_nibbles(packed)
+    yh = dequantize_groups(q, scales, group)
+    return sign_flip(inverse_rotate(yh, rot), signs)
+
+
+def attend_decode(q, k_packed, k_scales, v_packed, v_scales, length: int, signs, rot: int,
+                  group: int, sm_scale: float):
+    """Decode attention over the int4 cache: one query step.
+
+    [P1] "First, the 17%": K and V are dequantized and rotated back when
+    attention reads them; [P3]: that decode belongs inside the attention
+    kernel.  For every KV head h and each of its queries i, with
+    K_t, V_t = dequant_rotated_f64 of rows t < length of that head:
+        s_t = sm_scale <q_i, K_t>,  p = softmax(s),  o_i = sum_t p_t V_t,
+    in float64, rounded to fp16 at the end.
+
+    q: [H, nq, d] fp16; k_/v_packed [H, cap, d/2] uint8; k_/v_scales
+    [H, cap, d/g] float32.  Returns [H, nq, d] fp16.
+    """
+    q = np.asarray(q, dtype=np.float16).astype(np.float64)
+    h, nq, d = q.shape
+    out = np.empty((h, nq, d), dtype=np.float64)
+    for hh in range(h):
+        k = dequant_rotated_f64(k_packed[hh, :length], k_scales[hh, :length], signs, rot, group)
+        v = dequant_rotated_f64(v_packed[hh, :length], v_scales[hh, :length], signs, rot, group)
+        s = sm_scale * (q[hh] @ k.T)  # [nq, length]
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        out[hh] = p @ v
+    return out.astype(np.float16)

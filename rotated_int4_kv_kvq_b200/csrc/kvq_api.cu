@@ -1,6 +1,7 @@
 // kvq_api.cu -- the C ABI of libkvq: argument checks, TMA descriptors,
 // dispatch to the per-d kernels.  Declarations and contracts: include/kvq.h.
 #include <cuda.h>
+#include <cmath>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -279,6 +280,34 @@ kvq_status kvq_decode_step_windowed(const uint16_t* x_new, uint8_t* packed, floa
   cudaError_t e = d == 64    ? kvq::launch_window<64>(group, rot, W)
                   : d == 128 ? kvq::launch_window<128>(group, rot, W)
                              : kvq::launch_window<256>(group, rot, W);
+  return from_cuda(e);
+}
+
+kvq_status kvq_attend_decode(const uint16_t* q, const uint8_t* k_packed, const float* k_scales,
+                             const uint8_t* v_packed, const float* v_scales, int64_t n_kv_heads,
+                             int32_t n_q, int64_t cap, int64_t len, int32_t d, int32_t group,
+                             const int8_t* signs, kvq_rot rot, float sm_scale, uint16_t* out,
+                             kvq_stream stream) {
+  if (kvq_status s = check_shape(d, group, rot)) return s;
+  if (n_kv_heads < 0 || n_kv_heads > 65535 || n_q < 1 || n_q > 8 || cap < 1 || cap > kMaxRows ||
+      len < 1 || len > cap || !std::isfinite(sm_scale))
+    return KVQ_ERR_BAD_SIZE;
+  const int64_t ng = d / group;
+  if (n_kv_heads * cap * ng > kMaxRows || n_kv_heads * cap > kMaxRows) return KVQ_ERR_BAD_SIZE;
+  if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !signs || !out)
+    return KVQ_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_packed, 16) || !aligned(v_packed, 16) ||
+      !aligned(k_scales, 4) || !aligned(v_scales, 4))
+    return KVQ_ERR_MISALIGNED;
+  if (n_kv_heads == 0) return KVQ_OK;
+  DeviceInfo dev;
+  if (kvq_status s = device_info(&dev)) return s;
+  kvq::AttnLaunch A{q,   k_packed, k_scales, v_packed,     v_scales,
+                    out, signs,    n_kv_heads, cap,        len,
+                    n_q, sm_scale, dev.sm_count, reinterpret_cast<cudaStream_t>(stream)};
+  cudaError_t e = d == 64    ? kvq::launch_attn<64>(group, rot, A)
+                  : d == 128 ? kvq::launch_attn<128>(group, rot, A)
+                             : kvq::launch_attn<256>(group, rot, A);
   return from_cuda(e);
 }
 

@@ -7,5 +7,6 @@ template cudaError_t launch_inv<256>(int, int, const InvLaunch&);
 template cudaError_t launch_decode<256>(int, int, const DecodeLaunch&);
 template cudaError_t launch_decode_wide<256>(int, int, const DecodeWideLaunch&);
 template cudaError_t launch_window<256>(int, int, const WindowLaunch&);
+template cudaError_t launch_attn<256>(int, int, const AttnLaunch&);
 template cudaError_t read_status<256>(uint32_t*, bool);
 }  // namespace kvq

@@ -7,5 +7,6 @@ template cudaError_t launch_inv<64>(int, int, const InvLaunch&);
 template cudaError_t launch_decode<64>(int, int, const DecodeLaunch&);
 template cudaError_t launch_decode_wide<64>(int, int, const DecodeWideLaunch&);
 template cudaError_t launch_window<64>(int, int, const WindowLaunch&);
+template cudaError_t launch_attn<64>(int, int, const AttnLaunch&);
 template cudaError_t read_status<64>(uint32_t*, bool);
 }  // namespace kvq

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "kvq_codec.cuh"
+#include "kvq_attn.cuh"
 #include "kvq_wide.cuh"
 #include "kvq_launch.h"
 
@@ -236,6 +237,71 @@ cudaError_t window_one(const WindowLaunch& L) {
   return cudaGetLastError();
 }
 
+template <int D, int ROT, int NQ>
+cudaError_t attn_nq(int group, const AttnLaunch& L) {
+  constexpr auto kern = kvq_attn_kernel<D, ROT, NQ>;
+  constexpr int smem = attn_smem_bytes<D, NQ>();
+  int max_cluster;
+  {
+    static int maxc[kMaxDevices];
+    static std::mutex mu;
+    int dev;
+    cudaError_t e = current_device(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    if (maxc[dev] == 0) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      // clusters of up to 16 blocks where the device can co-schedule them
+      int c = 8;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+          cudaSuccess) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(16, 1, 1);
+        q.blockDim = dim3(kAttnThreads, 1, 1);
+        q.dynamicSmemBytes = smem;
+        int best = 0;
+        if (cudaOccupancyMaxPotentialClusterSize(&best, kern, &q) == cudaSuccess && best >= 8)
+          c = std::min(best, 16);
+      }
+      cudaGetLastError();
+      maxc[dev] = c;
+    }
+    max_cluster = maxc[dev];
+  }
+  // blocks per KV head (one cluster): about one staged chunk per warp, and no
+  // more than the SMs left per head (one resident block per SM)
+  constexpr int64_t per_block = int64_t(kAttnWarps) * kAttnChunk;
+  const int64_t by_len = (L.len + per_block - 1) / per_block;
+  const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
+  const int cl = int(std::max<int64_t>(
+      1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
+             L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(cl), unsigned(L.n_kv), 1);
+  cfg.blockDim = dim3(kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(cl);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
+template <int D, int ROT>
+cudaError_t attn_rot(int group, const AttnLaunch& L) {
+  if (L.nq <= 1) return attn_nq<D, ROT, 1>(group, L);
+  if (L.nq <= 2) return attn_nq<D, ROT, 2>(group, L);
+  if (L.nq <= 4) return attn_nq<D, ROT, 4>(group, L);
+  return attn_nq<D, ROT, 8>(group, L);
+}
+
 // Run Op<D, G, ROT>(launch) for the runtime (group, rot) pair.
 template <int D, template <int, int, int> class Op, class L>
 cudaError_t dispatch(int group, int rot, const L& l) {
@@ -302,6 +368,12 @@ cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L) {
 template <int D>
 cudaError_t launch_window(int group, int rot, const WindowLaunch& L) {
   return detail::dispatch<D, detail::WindowOp>(group, rot, L);
+}
+
+template <int D>
+cudaError_t launch_attn(int group, int rot, const AttnLaunch& L) {
+  return rot == kRotSRFT ? detail::attn_rot<D, kRotSRFT>(group, L)
+                         : detail::attn_rot<D, kRotSRHT>(group, L);
 }
 
 template <int D>

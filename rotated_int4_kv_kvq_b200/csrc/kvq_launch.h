@@ -63,6 +63,21 @@ struct WindowLaunch {
   cudaStream_t stream;
 };
 
+struct AttnLaunch {
+  const uint16_t* q;        // [n_kv][nq][d]
+  const uint8_t* k_packed;  // [n_kv][cap][d/2]
+  const float* k_scales;    // [n_kv][cap][d/g]
+  const uint8_t* v_packed;
+  const float* v_scales;
+  uint16_t* out;            // [n_kv][nq][d]
+  const int8_t* signs;
+  int64_t n_kv, cap, len;
+  int nq;
+  float sm_scale;
+  int sm_count;
+  cudaStream_t stream;
+};
+
 struct DecodeLaunch {
   const CUtensorMap* tmXn;  // x_new [n_heads][d], box {64, VPW}
   const CUtensorMap* tmQn;  // packed row pos of every head, box {d/2, VPW}
@@ -87,6 +102,9 @@ template <int D>
 cudaError_t launch_decode_wide(int group, int rot, const DecodeWideLaunch& L);
 template <int D>
 cudaError_t launch_window(int group, int rot, const WindowLaunch& L);
+// group is a runtime argument of the attention kernel.
+template <int D>
+cudaError_t launch_attn(int group, int rot, const AttnLaunch& L);
 // Reads (and optionally clears) the device status word of that translation
 // unit on the current device; the caller has synchronized the device.
 template <int D>

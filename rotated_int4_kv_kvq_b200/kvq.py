@@ -29,7 +29,7 @@ LIB_PATH = os.environ.get("KVQ_LIBRARY") or os.path.join(
 
 EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_rot_quant_fwd_lambda",
            "kvq_dequant_rot_inv_lambda", "kvq_decode_step", "kvq_decode_step_windowed",
-           "kvq_status_string", "kvq_device_status", "kvq_version")
+           "kvq_attend_decode", "kvq_status_string", "kvq_device_status", "kvq_version")
 
 
 class KVQError(RuntimeError):
@@ -57,6 +57,9 @@ def _load() -> ctypes.CDLL:
     lib.kvq_decode_step.restype = i32
     lib.kvq_decode_step_windowed.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, i32, p, i32, p]
     lib.kvq_decode_step_windowed.restype = i32
+    lib.kvq_attend_decode.argtypes = [p, p, p, p, p, i64, i32, i64, i64, i32, i32, p, i32,
+                                      ctypes.c_float, p, p]
+    lib.kvq_attend_decode.restype = i32
     lib.kvq_status_string.argtypes = [i32]
     lib.kvq_status_string.restype = ctypes.c_char_p
     lib.kvq_device_status.argtypes = [i32]
@@ -193,6 +196,32 @@ def kvq_decode_step_windowed(x_new: torch.Tensor, packed: torch.Tensor, scales: 
                                       pos, window, d, group, _ptr(signs), rot, _stream(stream))
     _raise("kvq_decode_step_windowed", st)
     return kv
+
+
+def kvq_attend_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.Tensor,
+                      v_packed: torch.Tensor, v_scales: torch.Tensor, length: int,
+                      signs: torch.Tensor, rot: int, group: int, sm_scale: float | None = None,
+                      out: torch.Tensor | None = None, stream=None):
+    """Decode attention over the int4 cache: q [H, nq, d] fp16 against
+    rows [0, length) of the K/V caches [H, cap, d/2] (+ scales); returns
+    out [H, nq, d] fp16.  sm_scale defaults to 1/sqrt(d)."""
+    h, nq, d = q.shape
+    cap = k_packed.shape[1]
+    _check(q, "q", torch.float16, (h, nq, d))
+    for name, t in (("k_packed", k_packed), ("v_packed", v_packed)):
+        _check(t, name, torch.uint8, (h, cap, d // 2))
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _check(t, name, torch.float32, (h, cap, d // group))
+    _check(signs, "signs", torch.int8, (d,))
+    if out is None:
+        out = torch.empty((h, nq, d), dtype=torch.float16, device=q.device)
+    _check(out, "out", torch.float16, (h, nq, d))
+    scale = float(sm_scale) if sm_scale is not None else d ** -0.5
+    st = lib.kvq_attend_decode(_ptr(q), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+                               _ptr(v_scales), h, nq, cap, length, d, group, _ptr(signs), rot,
+                               scale, _ptr(out), _stream(stream))
+    _raise("kvq_attend_decode", st)
+    return out
 
 
 def kvq_device_status(clear: bool = True) -> int:

@@ -128,3 +128,23 @@ def test_lambda_host_checks(kvq):
     assert inv(A, A, 10, 64, 16, A, A, 0, A, None) == 3
     assert fwd(A, 0, 64, 32, A, A, 0, A, A, None) == 0
     assert inv(A, A, 0, 64, 32, A, A, 1, A, None) == 0
+
+
+def test_attend_host_checks(kvq):
+    lib = kvq.lib
+    att = lib.kvq_attend_decode
+    # (q, kp, ks, vp, vs, n_kv, n_q, cap, len, d, g, signs, rot, sm_scale, out, stream)
+    assert att(A, A, A, A, A, 2, 4, 16, 10, 96, 32, A, 0, 0.125, A, None) == 2
+    assert att(A, A, A, A, A, 2, 4, 16, 10, 64, 16, A, 0, 0.125, A, None) == 3
+    assert att(A, A, A, A, A, 2, 4, 16, 10, 64, 32, A, 7, 0.125, A, None) == 5
+    assert att(A, A, A, A, A, 2, 0, 16, 10, 64, 32, A, 0, 0.125, A, None) == 7
+    assert att(A, A, A, A, A, 2, 9, 16, 10, 64, 32, A, 0, 0.125, A, None) == 7
+    assert att(A, A, A, A, A, 2, 4, 16, 0, 64, 32, A, 0, 0.125, A, None) == 7
+    assert att(A, A, A, A, A, 2, 4, 16, 17, 64, 32, A, 0, 0.125, A, None) == 7
+    assert att(A, A, A, A, A, 70000, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 7
+    assert att(A, A, A, A, A, 2, 4, 16, 10, 64, 32, A, 0, float("inf"), A, None) == 7
+    assert att(A, None, A, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 1
+    assert att(A, A, A, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, None, None) == 1
+    assert att(A + 8, A, A, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 4
+    assert att(A, A, A + 2, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 4
+    assert att(A, A, A, A, A, 0, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 0

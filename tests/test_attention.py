@@ -1,0 +1,85 @@
+"""Decode attention over the int4 cache (needs a B200): kvq_attend_decode
+against the oracle's attend_decode (float64 softmax over the exactly
+dequantized, inverse-rotated K and V).  The cache rows are written by the
+library's own forward kernel; rows beyond `len` hold garbage that must not
+leak into the result."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.kvq_oracle as O
+from rotated_int4_kv_kvq_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+OUT_RTOL = 2e-3  # of the largest output element of the row (fp16 rounding: 2^-11)
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from rotated_int4_kv_kvq_b200 import kvq as mod
+    return mod
+
+
+def make_cache(kvq, heads, cap, d, group, rot, signs, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    out = []
+    for _ in range(2):  # K, V
+        x = (torch.randn((heads * cap, d), generator=g, device="cuda") * 2).half()
+        x[:, 7] *= 15  # an outlier channel
+        p, s = kvq.kvq_rot_quant_fwd(x, signs, rot, group)
+        out += [p.reshape(heads, cap, -1), s.reshape(heads, cap, -1)]
+    q = (torch.randn((heads, 8, d), generator=g, device="cuda")).half()
+    return out, q
+
+
+def run_case(kvq, d, group, rot, heads, nq, length, sm_scale=None, seed=0):
+    cap = length + 5
+    signs_np = W.make_signs(d)
+    signs = torch.from_numpy(signs_np).cuda()
+    (kp, ks, vp, vs), qall = make_cache(kvq, heads, cap, d, group, rot, signs, seed)
+    # garbage beyond len
+    kp[:, length:] = 0x77
+    vp[:, length:] = 0x17
+    ks[:, length:] = 1e30
+    vs[:, length:] = 1e30
+    q = qall[:, :nq].contiguous()
+    scale = d ** -0.5 if sm_scale is None else sm_scale
+    out = kvq.kvq_attend_decode(q, kp, ks, vp, vs, length, signs, rot, group, scale)
+    torch.cuda.synchronize()
+    assert kvq.kvq_device_status() == 0
+    ref = O.attend_decode(q.cpu().numpy(), kp.cpu().numpy(), ks.cpu().numpy(), vp.cpu().numpy(),
+                          vs.cpu().numpy(), length, signs_np, rot, group, scale)
+    got = out.cpu().numpy().astype(np.float64)
+    r = ref.astype(np.float64)
+    tol = OUT_RTOL * np.abs(r).max(axis=2, keepdims=True) + 1e-6
+    err = np.abs(got - r)
+    assert np.all(err <= tol), f"max err {(err / tol).max():.3g} x tol"
+    return got
+
+
+@pytest.mark.parametrize("d,group", [(64, 32), (64, 64), (128, 32), (128, 128), (256, 64),
+                                     (256, 256)])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("nq,length", [(1, 1), (4, 7), (1, 300), (2, 333), (4, 2500),
+                                       (8, 1000), (6, 97)])
+def test_attention_parity(kvq, d, group, rot, nq, length):
+    run_case(kvq, d, group, rot, heads=2, nq=nq, length=length, seed=d + length + nq)
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+def test_attention_sharp_and_flat(kvq, rot):
+    """sm_scale 0: the mean of V; a large scale: close to one-hot weights."""
+    run_case(kvq, 256, 256, rot, heads=1, nq=4, length=513, sm_scale=0.0, seed=3)
+    run_case(kvq, 128, 32, rot, heads=3, nq=2, length=200, sm_scale=4.0, seed=4)
+
+
+def test_attention_gemma_shape(kvq):
+    """Gemma-3-1B-like layer: 1 KV head, 4 queries, d = g = 256, 4096 rows."""
+    run_case(kvq, 256, 256, O.SRFT, heads=1, nq=4, length=4096, seed=9)
+
+
+def test_attention_many_heads(kvq):
+    """SmolLM2-1.7B-like layer: 32 KV heads, one query each, d = g = 64."""
+    run_case(kvq, 64, 64, O.SRFT, heads=32, nq=1, length=1024, seed=10)

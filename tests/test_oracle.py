@@ -276,6 +276,55 @@ def check_lambda(rot=O.SRFT, d=64, group=32):
     assert np.array_equal(xi, xr / lam)
 
 
+def _attn_case(rot, d=64, group=32, h=2, nq=3, n=9, seed=13):
+    rng = np.random.default_rng(seed)
+    signs = W.make_signs(d)
+    kx = (rng.standard_normal((h * n, d)) * 2).astype(np.float16)
+    vx = (rng.standard_normal((h * n, d)) * 2).astype(np.float16)
+    kp, ks = O.rot_quant_fwd(kx, signs, rot, group)
+    vp, vs = O.rot_quant_fwd(vx, signs, rot, group)
+    q = (rng.standard_normal((h, nq, d))).astype(np.float16)
+    return (signs, q, kp.reshape(h, n, -1), ks.reshape(h, n, -1), vp.reshape(h, n, -1),
+            vs.reshape(h, n, -1))
+
+
+def check_attention(rot=O.SRFT, d=64, group=32):
+    """Decode attention over the int4 cache: one key gives its value; a zero
+    softmax scale gives the mean value; a large scale with a unique best key
+    gives that key's value; and the whole result equals the same attention
+    computed in the rotated domain (scores <R D q, y_hat_K>, values
+    D R^T sum_t p_t y_hat_V,t), a different route through R."""
+    signs, q, kp, ks, vp, vs = _attn_case(rot, d, group)
+    h, nq, _ = q.shape
+    n = kp.shape[1]
+    v64 = [O.dequant_rotated_f64(vp[i], vs[i], signs, rot, group) for i in range(h)]
+    one = O.attend_decode(q, kp, ks, vp, vs, 1, signs, rot, group, 0.125)
+    assert np.array_equal(one, np.repeat(np.stack([v[0] for v in v64])[:, None], nq, 1)
+                          .astype(np.float16))
+    flat = O.attend_decode(q, kp, ks, vp, vs, n, signs, rot, group, 0.0)
+    assert np.array_equal(flat, np.repeat(np.stack([v.mean(0) for v in v64])[:, None], nq, 1)
+                          .astype(np.float16))
+    k64 = [O.dequant_rotated_f64(kp[i], ks[i], signs, rot, group) for i in range(h)]
+    sc = np.stack([q[i].astype(np.float64) @ k64[i].T for i in range(h)])  # [h, nq, n]
+    order = np.sort(sc, axis=2)
+    if np.all(order[..., -1] - order[..., -2] > 1e-3):
+        sharp = O.attend_decode(q, kp, ks, vp, vs, n, signs, rot, group, 1e7)
+        best = sc.argmax(axis=2)
+        ref = np.stack([[v64[i][best[i, j]] for j in range(nq)] for i in range(h)])
+        assert np.array_equal(sharp, ref.astype(np.float16))
+    got = O.attend_decode(q, kp, ks, vp, vs, n, signs, rot, group, 0.3)
+    for i in range(h):
+        qr = O.rotate(O.sign_flip(q[i].astype(np.float64), signs), rot)  # [nq, d]
+        yk = O.dequantize_groups(O.unpack_nibbles(kp[i]), ks[i], group)
+        yv = O.dequantize_groups(O.unpack_nibbles(vp[i]), vs[i], group)
+        s_ = 0.3 * (qr @ yk.T)
+        p_ = np.exp(s_ - s_.max(axis=1, keepdims=True))
+        p_ /= p_.sum(axis=1, keepdims=True)
+        o_ = O.sign_flip(O.inverse_rotate(p_ @ yv, rot), signs)
+        assert np.array_equal(got[i], o_.astype(np.float16)) or \
+            np.abs(got[i].astype(np.float64) - o_).max() <= 2.0 ** -10 * np.abs(o_).max()
+
+
 # ------------------------------------------------------------------ tests ---
 
 @pytest.mark.parametrize("d", [2, 4, 8, 64, 128, 256])
@@ -364,6 +413,12 @@ def test_decode_windowed_matches_plain_decode(rot, window):
 @pytest.mark.parametrize("d,group", [(64, 32), (256, 256)])
 def test_lambda_hook(rot, d, group):
     check_lambda(rot, d, group)
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("d,group", [(64, 32), (256, 256)])
+def test_attention(rot, d, group):
+    check_attention(rot, d, group)
 
 
 def test_granularity_monotone():
@@ -500,6 +555,14 @@ def _mut_lambda_after_rotation(x_fp16, signs, rot, lam=None):
     return y
 
 
+def _mut_attn_fp16_keys(packed, scales, signs, rot, group):
+    # keys and values rounded to fp16 first (a different definition)
+    q = O.unpack_nibbles(packed)
+    yh = O.dequantize_groups(q, scales, group)
+    x = O.sign_flip(O.inverse_rotate(yh, rot), signs)
+    return x.astype(np.float16).astype(np.float64) * (1 + 2.0 ** -9)
+
+
 def _mut_inverse_no_transpose(y, rot):
     return np.asarray(y, np.float64) @ O.rotation_matrix(y.shape[-1], rot).T
 
@@ -528,6 +591,7 @@ MUTATIONS = [
     ("decode_step_windowed", _mut_window_flush_early,
      [lambda: check_decode_windowed(window=4)]),
     ("rotated_values", _mut_lambda_after_rotation, [check_lambda]),
+    ("dequant_rotated_f64", _mut_attn_fp16_keys, [check_attention]),
 ]
 
 
