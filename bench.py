@@ -565,6 +565,31 @@ def run_suite(kvq, dev):
                         "us": us, "algo_gbs": algo / (us * 1e-6) / 1e9,
                         "fp16_gbs": n * d * 2 / (us * 1e-6) / 1e9,
                         "vec_per_s": n / (us * 1e-6), "frac": algo / (us * 1e-6) / 1e9 / peak})
+                if g == d and rot == kvq.SRFT:  # other code widths on the same workload
+                    for bits in ((3, 6, 8) if d >= 128 else (6, 8)):
+                        pb = torch.empty((n, d * bits // 8), dtype=torch.uint8, device=dev)
+                        ab = n * (2 * d + d * bits // 8 + 4 * (d // g))
+                        for _ in range(3):
+                            kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
+                            kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
+                        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                        tf = ti = 0.0
+                        for _ in range(steps):
+                            e[0].record()
+                            kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
+                            e[1].record()
+                            kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
+                            e[2].record()
+                            torch.cuda.synchronize()
+                            tf += e[0].elapsed_time(e[1])
+                            ti += e[1].elapsed_time(e[2])
+                        for name, ms in (("fwd", tf), ("inv", ti)):
+                            us = 1e3 * ms / steps
+                            res.setdefault("bits", []).append({
+                                "d": d, "group": g, "rot": "srft", "bits": bits, "dir": name,
+                                "us": us, "algo_gbs": ab / (us * 1e-6) / 1e9,
+                                "frac": ab / (us * 1e-6) / 1e9 / peak})
+                        del pb
                 if g == d:  # the per-channel lambda hook on the same workload
                     lam = torch.exp(0.5 * torch.randn(d, generator=torch.Generator().manual_seed(d)))
                     lam = lam.to(dev)

@@ -79,7 +79,8 @@ typedef enum {
   KVQ_ERR_CUDA = 6,           /* CUDA runtime error while enqueueing        */
   KVQ_ERR_BAD_SIZE = 7,       /* negative or too large count / position     */
   KVQ_ERR_DEVICE_TIMEOUT = 8, /* a kernel gave up waiting for its own copy  */
-  KVQ_ERR_UNSUPPORTED_DEVICE = 9 /* device is not compute capability 10.0  */
+  KVQ_ERR_UNSUPPORTED_DEVICE = 9, /* device is not compute capability 10.0 */
+  KVQ_ERR_BAD_BITS = 10       /* code width not 3 (d >= 128), 4, 6 or 8     */
 } kvq_status;
 
 /*
@@ -139,6 +140,31 @@ kvq_status kvq_dequant_rot_inv_lambda(const uint8_t *packed, const float *scales
                                       const int8_t *signs, const float *lambda,
                                       kvq_rot rot, uint16_t *out,
                                       kvq_stream stream);
+
+/*
+ * Forward and inverse steps with another code width b ("Quantization Speed
+ * Is Often a Kernel Problem": "6-bit and 8-bit are lossless; 3-bit is worse";
+ * "Chapter 25 - Quantization: The Hardware View", sample quantizer:
+ * qmax = 2^(b-1) - 1):
+ *   s_j = max|y_i| / (2^(b-1) - 1), q_i = round_half_even(y_i / s_j);
+ *   packed row of a vector: d*b/8 bytes, a little-endian bitstream in which
+ *   code i occupies bits [b i, b i + b) as b-bit two's complement (for b = 4
+ *   this is the nibble layout above).
+ *   bits    3 (d >= 128 only: a d = 64 row would be 24 bytes), 4, 6 or 8;
+ *           anything else -> KVQ_ERR_BAD_BITS
+ *   packed  [n_vec][d*bits/8] uint8, 16-byte aligned
+ *   other arguments as in kvq_rot_quant_fwd / kvq_dequant_rot_inv.
+ */
+kvq_status kvq_rot_quant_fwd_bits(const uint16_t *x, int64_t n_vec, int32_t d,
+                                  int32_t group, int32_t bits,
+                                  const int8_t *signs, kvq_rot rot,
+                                  uint8_t *packed, float *scales,
+                                  kvq_stream stream);
+kvq_status kvq_dequant_rot_inv_bits(const uint8_t *packed, const float *scales,
+                                    int64_t n_vec, int32_t d, int32_t group,
+                                    int32_t bits, const int8_t *signs,
+                                    kvq_rot rot, uint16_t *out,
+                                    kvq_stream stream);
 
 /*
  * Decode step for one head-major cache, one launch ("A scene" and "First,

@@ -51,6 +51,9 @@ Readings where the pages are silent:
 * R7 groups are runs of g consecutive coordinates of the rotated, packed y.
 * R8 inverse: x_hat = D R^T y_hat with y_hat = s q in float64, rounded to
   float16 (round to nearest even) at the end.
+* R16 other code widths b: qmax = 2^(b-1) - 1 ([P5] formula), codes in a
+  little-endian bitstream per vector (code i at bits [b i, b i + b)); b = 4
+  is the nibble layout of R6.
 
 Parity pins for every function live in ``tests/test_oracle.py``.
 """
@@ -70,7 +73,7 @@ __all__ = [
     "rotate", "inverse_rotate", "quantize_groups", "dequantize_groups",
     "pack_nibbles", "unpack_nibbles", "rot_quant_fwd", "dequant_rot_inv",
     "rotated_values", "near_tie_distance", "decode_step", "decode_step_windowed",
-    "dequant_rotated_f64", "attend_decode",
+    "dequant_rotated_f64", "attend_decode", "pack_codes", "unpack_codes",
 ]
 
 
@@ -152,26 +155,29 @@ def inverse_rotate(y, rot: int) -> np.ndarray:
     return y @ r
 
 
-def quantize_groups(y, group: int):
-    """Per-group symmetric absmax int4 quantization (readings R4, R5, R7).
+def quantize_groups(y, group: int, bits: int = 4):
+    """Per-group symmetric absmax quantization (readings R4, R5, R7).
 
     [P1] "Fusing four steps...": one abs-max per group of consecutive values.
     [P5] sample quantizer: scale = amax / qmax, q = clamp(round(y/scale),
-    -qmax-1, qmax) with qmax = 7.  [P4]: the rounding error is at most s/2.
+    -qmax-1, qmax) with qmax = 2**(bits-1) - 1 (7 for int4; the pages' other
+    widths, [P1] "6-bit and 8-bit are lossless; 3-bit is worse", use the same
+    formula).  [P4]: the rounding error is at most s/2.
 
     Returns (q int8 [n, d], s float32 [n, d/group]).
     """
+    qmax = 2 ** (bits - 1) - 1
     y32 = np.asarray(y, dtype=np.float64).astype(np.float32)
     n, d = y32.shape
     if group <= 0 or d % group:
         raise ValueError("group must divide d")
     yg = y32.reshape(n, d // group, group)
     m = np.abs(yg).max(axis=2)  # exact in float32
-    s = (m / np.float32(QMAX)).astype(np.float32)  # one IEEE fp32 division
+    s = (m / np.float32(qmax)).astype(np.float32)  # one IEEE fp32 division
     safe = np.where(s > 0, s, np.float32(1.0))
     t = (yg / safe[..., None]).astype(np.float32)  # IEEE fp32 division
     t = np.where(s[..., None] > 0, t, np.float32(0.0))
-    q = np.clip(np.rint(t), QMIN, QMAX)  # rint: round half to even
+    q = np.clip(np.rint(t), -qmax - 1, qmax)  # rint: round half to even
     return q.astype(np.int8).reshape(n, d), s
 
 
@@ -192,6 +198,33 @@ def pack_nibbles(q) -> np.ndarray:
         raise ValueError("codes outside [-8, 7]")
     nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
     return (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+
+
+def pack_codes(q, bits: int) -> np.ndarray:
+    """b-bit two's complement codes as one little-endian bitstream per row:
+    code i occupies bits [b i, b i + b) and byte k holds bits [8k, 8k + 8)
+    (reading R16; for b = 4 this is exactly pack_nibbles' layout)."""
+    q = np.asarray(q)
+    n, d = q.shape
+    if (d * bits) % 8:
+        raise ValueError("row does not fill whole bytes")
+    lo, hi = -(2 ** (bits - 1)), 2 ** (bits - 1) - 1
+    if q.min(initial=0) < lo or q.max(initial=0) > hi:
+        raise ValueError("codes out of range")
+    u = (q.astype(np.int32) & ((1 << bits) - 1)).astype(np.uint32)
+    bitpos = np.arange(bits, dtype=np.uint32)
+    stream = ((u[..., None] >> bitpos) & 1).astype(np.uint8).reshape(n, d * bits)
+    return np.packbits(stream, axis=1, bitorder="little")
+
+
+def unpack_codes(packed, bits: int) -> np.ndarray:
+    """Inverse of pack_codes: sign-extended int8 codes [n, 8 * bytes / b]."""
+    p = np.asarray(packed, dtype=np.uint8)
+    n, nb = p.shape
+    d = nb * 8 // bits
+    stream = np.unpackbits(p, axis=1, bitorder="little")[:, : d * bits].reshape(n, d, bits)
+    u = (stream.astype(np.int32) << np.arange(bits, dtype=np.int32)).sum(axis=2)
+    return np.where(u >= 2 ** (bits - 1), u - 2 ** bits, u).astype(np.int8)
 
 
 def unpack_nibbles(packed) -> np.ndarray:
@@ -216,7 +249,7 @@ def rotated_values(x_fp16, signs, rot: int, lam=None) -> np.ndarray:
     return rotate(sign_flip(x, signs), rot)
 
 
-def rot_quant_fwd(x_fp16, signs, rot: int, group: int, lam=None):
+def rot_quant_fwd(x_fp16, signs, rot: int, group: int, lam=None, bits: int = 4):
     """Forward step: sign flip -> rotation -> per-group absmax int4 -> pack.
 
     [P1] "First, the 17%" and "Fusing four steps...": the forward kernel does
@@ -227,19 +260,20 @@ def rot_quant_fwd(x_fp16, signs, rot: int, group: int, lam=None):
     an input here, applied before the sign flip and the rotation.
     """
     y = rotated_values(x_fp16, signs, rot, lam)
-    q, s = quantize_groups(y, group)
-    return pack_nibbles(q), s
+    q, s = quantize_groups(y, group, bits)
+    return (pack_nibbles(q) if bits == 4 else pack_codes(q, bits)), s
 
 
-def dequant_rot_inv(packed, scales, signs, rot: int, group: int, lam=None) -> np.ndarray:
+def dequant_rot_inv(packed, scales, signs, rot: int, group: int, lam=None,
+                    bits: int = 4) -> np.ndarray:
     """Inverse step: unpack -> y_hat = s q -> u = R^T y_hat -> x_hat = D u.
 
     [P1] "First, the 17%": dequantized and rotated back when attention reads
     it.  The float64 result is rounded to float16 once (reading R8).  With
     `lam`, channel i is divided by lam[i] before that rounding (the inverse of
-    rot_quant_fwd's scaling).
+    rot_quant_fwd's scaling).  `bits`: the code width of rot_quant_fwd.
     """
-    q = unpack_nibbles(packed)
+    q = unpack_nibbles(packed) if bits == 4 else unpack_codes(packed, bits)
     yh = dequantize_groups(q, scales, group)
     u = sign_flip(inverse_rotate(yh, rot), signs)
     if lam is not None:

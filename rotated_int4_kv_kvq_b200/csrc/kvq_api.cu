@@ -103,6 +103,16 @@ bool map_x(CUtensorMap* m, const void* base, int d, uint64_t rows, uint64_t pitc
 }
 
 // packed-code rows [rows][d/2] with row pitch `pitch` bytes, box {d/2, VPW}.
+// codes of other widths: rows of d*bits/8 bytes, box {d*bits/8, VPW}, no swizzle.
+bool map_qb(CUtensorMap* m, const void* base, int d, int bits, uint64_t rows) {
+  const uint64_t qp = uint64_t(d) * uint64_t(bits) / 8;
+  const uint64_t dims[2] = {qp, rows};
+  const uint64_t strides[1] = {qp};
+  const uint32_t box[2] = {uint32_t(qp), uint32_t(vpw_of(d))};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool map_q(CUtensorMap* m, const void* base, int d, uint64_t rows, uint64_t pitch) {
   const uint64_t dims[2] = {uint64_t(d / 2), rows};
   const uint64_t strides[1] = {pitch};
@@ -122,10 +132,15 @@ kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR
 
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
 
+bool bits_ok(int32_t d, int32_t bits) {
+  return bits == 4 || bits == 6 || bits == 8 || (bits == 3 && d >= 128);
+}
+
 kvq_status rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
                          const int8_t* signs, const float* lambda, kvq_rot rot, uint8_t* packed,
-                         float* scales, kvq_stream stream) {
+                         float* scales, kvq_stream stream, int32_t bits = 4) {
   if (kvq_status s = check_shape(d, group, rot)) return s;
+  if (!bits_ok(d, bits)) return KVQ_ERR_BAD_BITS;
   if (n_vec < 0 || n_vec > kMaxRows) return KVQ_ERR_BAD_SIZE;
   if (!x || !signs || !packed || !scales) return KVQ_ERR_NULL;
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 16) ||
@@ -136,9 +151,10 @@ kvq_status rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t gr
   if (kvq_status s = device_info(&dev)) return s;
   CUtensorMap tmX, tmQ;
   if (!map_x(&tmX, x, d, uint64_t(n_vec), uint64_t(2 * d)) ||
-      !map_q(&tmQ, packed, d, uint64_t(n_vec), uint64_t(d / 2)))
+      !(bits == 4 ? map_q(&tmQ, packed, d, uint64_t(n_vec), uint64_t(d / 2))
+                  : map_qb(&tmQ, packed, d, bits, uint64_t(n_vec))))
     return KVQ_ERR_CUDA;
-  kvq::FwdLaunch L{&tmX, &tmQ, signs, lambda, scales, n_vec, dev.sm_count,
+  kvq::FwdLaunch L{&tmX, &tmQ, signs, lambda, bits, scales, n_vec, dev.sm_count,
                    reinterpret_cast<cudaStream_t>(stream)};
   cudaError_t e = d == 64    ? kvq::launch_fwd<64>(group, rot, L)
                   : d == 128 ? kvq::launch_fwd<128>(group, rot, L)
@@ -148,8 +164,9 @@ kvq_status rot_quant_fwd(const uint16_t* x, int64_t n_vec, int32_t d, int32_t gr
 
 kvq_status dequant_rot_inv(const uint8_t* packed, const float* scales, int64_t n_vec, int32_t d,
                            int32_t group, const int8_t* signs, const float* lambda, kvq_rot rot,
-                           uint16_t* out, kvq_stream stream) {
+                           uint16_t* out, kvq_stream stream, int32_t bits = 4) {
   if (kvq_status s = check_shape(d, group, rot)) return s;
+  if (!bits_ok(d, bits)) return KVQ_ERR_BAD_BITS;
   if (n_vec < 0 || n_vec > kMaxRows || n_vec * (d / group) > kMaxRows) return KVQ_ERR_BAD_SIZE;
   if (!packed || !scales || !signs || !out) return KVQ_ERR_NULL;
   if (!aligned(packed, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
@@ -159,11 +176,12 @@ kvq_status dequant_rot_inv(const uint8_t* packed, const float* scales, int64_t n
   DeviceInfo dev;
   if (kvq_status s = device_info(&dev)) return s;
   CUtensorMap tmQ, tmS, tmX;
-  if (!map_q(&tmQ, packed, d, uint64_t(n_vec), uint64_t(d / 2)) ||
+  if (!(bits == 4 ? map_q(&tmQ, packed, d, uint64_t(n_vec), uint64_t(d / 2))
+                  : map_qb(&tmQ, packed, d, bits, uint64_t(n_vec))) ||
       !map_s(&tmS, scales, d, group, uint64_t(n_vec) * uint64_t(d / group)) ||
       !map_x(&tmX, out, d, uint64_t(n_vec), uint64_t(2 * d)))
     return KVQ_ERR_CUDA;
-  kvq::InvLaunch L{&tmQ, &tmS, &tmX, signs, lambda, n_vec, dev.sm_count,
+  kvq::InvLaunch L{&tmQ, &tmS, &tmX, signs, lambda, bits, n_vec, dev.sm_count,
                    reinterpret_cast<cudaStream_t>(stream)};
   cudaError_t e = d == 64    ? kvq::launch_inv<64>(group, rot, L)
                   : d == 128 ? kvq::launch_inv<128>(group, rot, L)
@@ -200,6 +218,18 @@ kvq_status kvq_dequant_rot_inv_lambda(const uint8_t* packed, const float* scales
                                       kvq_stream stream) {
   if (!lambda) return KVQ_ERR_NULL;
   return dequant_rot_inv(packed, scales, n_vec, d, group, signs, lambda, rot, out, stream);
+}
+
+kvq_status kvq_rot_quant_fwd_bits(const uint16_t* x, int64_t n_vec, int32_t d, int32_t group,
+                                  int32_t bits, const int8_t* signs, kvq_rot rot, uint8_t* packed,
+                                  float* scales, kvq_stream stream) {
+  return rot_quant_fwd(x, n_vec, d, group, signs, nullptr, rot, packed, scales, stream, bits);
+}
+
+kvq_status kvq_dequant_rot_inv_bits(const uint8_t* packed, const float* scales, int64_t n_vec,
+                                    int32_t d, int32_t group, int32_t bits, const int8_t* signs,
+                                    kvq_rot rot, uint16_t* out, kvq_stream stream) {
+  return dequant_rot_inv(packed, scales, n_vec, d, group, signs, nullptr, rot, out, stream, bits);
 }
 
 kvq_status kvq_decode_step(const uint16_t* x_new, uint8_t* packed, float* scales,
@@ -323,6 +353,7 @@ const char* kvq_status_string(kvq_status s) {
     case KVQ_ERR_BAD_SIZE: return "count or position out of range";
     case KVQ_ERR_DEVICE_TIMEOUT: return "a kernel timed out waiting for its own copy";
     case KVQ_ERR_UNSUPPORTED_DEVICE: return "device is not compute capability 10.0 (sm_100a)";
+    case KVQ_ERR_BAD_BITS: return "bits must be 3 (d >= 128), 4, 6 or 8";
   }
   return "unknown status";
 }

@@ -42,20 +42,25 @@ constexpr int kThreads = kWarps * 32;
 //           pair_join_fwd); both halves are in natural y order.
 constexpr int kLayFull = 0, kLayHalf = 1, kLayQuarter = 2;
 
-template <int D_, int ROT_, int TPV_>
+template <int D_, int ROT_, int TPV_, int BITS_ = 4>
 struct Cfg {
   static constexpr int D = D_;
   static constexpr int ROT = ROT_;
   static constexpr int TPV = TPV_;
+  static constexpr int BITS = BITS_;       // code width
   static constexpr int VPW = 32 / TPV;     // vectors per warp tile
   static constexpr int E = D / TPV;        // reals per thread
   static constexpr int P = E / 2;          // float pairs per thread
   static constexpr int NW = E / 2;         // fp16-pair words per thread
-  static constexpr int NQ = E / 8;         // packed-code words per thread
+  static constexpr int NQ = E * BITS / 32;  // packed-code words per thread
   static constexpr int XTILE = VPW * D * 2;  // fp16 tile bytes
-  static constexpr int QTILE = VPW * D / 2;  // code tile bytes
+  static constexpr int QTILE = VPW * D * BITS / 8;  // code tile bytes
+  // shared-memory stride of a code tile: whole KiB, so that the swizzled
+  // tiles placed after it keep the 1024-byte alignment TMA swizzling needs
+  static constexpr int QSTRIDE = (QTILE + 1023) / 1024 * 1024;
   static constexpr int SLAB = VPW * 128;   // one 64-column fp16 slab
-  static constexpr int QP = D / 2;         // code row pitch in bytes
+  static constexpr int QP = D * BITS / 8;  // code row pitch in bytes
+  static constexpr int QMAX = (1 << (BITS - 1)) - 1;
   static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
   // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
   // takes Yin = KAPPA_INV * y_hat.  SRFT (Y = packed rfft with X_0, X_{d/2}
@@ -70,8 +75,10 @@ struct Cfg {
   static constexpr double KAPPA_INV_D =
       ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : 1.0 / const_sqrt(2.0 * D);
   static constexpr float KAPPA_INV = float(KAPPA_INV_D);
-  static constexpr float KAPPA7 = float(KAPPA_FWD_D / 7.0);
+  static constexpr float KAPPA7 = float(KAPPA_FWD_D / QMAX);  // stored scale = m * KAPPA7
   static_assert(D % 64 == 0 && (TPV == 1 || TPV == 2), "shape");
+  static_assert(BITS == 3 || BITS == 4 || BITS == 6 || BITS == 8, "code width");
+  static_assert(BITS == 4 || QP % 16 == 0, "code rows must be whole 16-byte chunks");
 };
 
 template <int D>
@@ -206,25 +213,49 @@ __device__ __forceinline__ int code_chunk(int t, int lc) {
   return global_y<C>(t, 32 * lc) / 32;
 }
 
+// Codes of the thread's runs of 32 consecutive y coordinates: 4-bit tiles
+// are swizzled 16-byte chunks; other widths are plain rows of QP bytes, a run
+// of 32 codes being BITS whole words.
+template <class C>
+__device__ __forceinline__ uint32_t run_byte(int t, int run) {
+  return uint32_t(global_y<C>(t, 32 * run) * C::BITS / 8);
+}
+
 template <class C>
 __device__ __forceinline__ void load_codes(uint32_t tile, int row, int t, uint32_t (&qw)[C::NQ]) {
+  if constexpr (C::BITS == 4) {
 #pragma unroll
-  for (int c = 0; c < C::NQ / 4; ++c) {
-    const uint4 v = lds128(tile + swq<C::QP>(row, code_chunk<C>(t, c)));
-    qw[4 * c] = v.x;
-    qw[4 * c + 1] = v.y;
-    qw[4 * c + 2] = v.z;
-    qw[4 * c + 3] = v.w;
+    for (int c = 0; c < C::NQ / 4; ++c) {
+      const uint4 v = lds128(tile + swq<C::QP>(row, code_chunk<C>(t, c)));
+      qw[4 * c] = v.x;
+      qw[4 * c + 1] = v.y;
+      qw[4 * c + 2] = v.z;
+      qw[4 * c + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < C::E / 32; ++r)
+#pragma unroll
+      for (int k = 0; k < C::BITS; ++k)
+        qw[r * C::BITS + k] = lds32(tile + uint32_t(row * C::QP) + run_byte<C>(t, r) + 4u * k);
   }
 }
 
 template <class C>
 __device__ __forceinline__ void store_codes(uint32_t tile, int row, int t,
                                             const uint32_t (&qw)[C::NQ]) {
+  if constexpr (C::BITS == 4) {
 #pragma unroll
-  for (int c = 0; c < C::NQ / 4; ++c)
-    sts128(tile + swq<C::QP>(row, code_chunk<C>(t, c)), qw[4 * c], qw[4 * c + 1], qw[4 * c + 2],
-           qw[4 * c + 3]);
+    for (int c = 0; c < C::NQ / 4; ++c)
+      sts128(tile + swq<C::QP>(row, code_chunk<C>(t, c)), qw[4 * c], qw[4 * c + 1],
+             qw[4 * c + 2], qw[4 * c + 3]);
+  } else {
+#pragma unroll
+    for (int r = 0; r < C::E / 32; ++r)
+#pragma unroll
+      for (int k = 0; k < C::BITS; ++k)
+        sts32(tile + uint32_t(row * C::QP) + run_byte<C>(t, r) + 4u * k, qw[r * C::BITS + k]);
+  }
 }
 
 // ------------------------------------------------------ forward rotation ---
@@ -523,9 +554,27 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
   const f2 magic = mk2(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) {
-    const float inv = m[g] > 0.0f ? __fdiv_rn(7.0f, m[g]) : 0.0f;
+    const float inv = m[g] > 0.0f ? __fdiv_rn(float(C::QMAX), m[g]) : 0.0f;
     sc[g] = m[g] * C::KAPPA7;
     const f2 inv2 = mk2(inv, inv);
+    if constexpr (C::BITS != 4) {
+      // runs of 32 codes -> BITS words of a little-endian bitstream
+#pragma unroll
+      for (int r = 0; r < GP / 16; ++r) {
+        uint32_t f[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const f2 v = Y[g * GP + 16 * r + i];
+          f[2 * i] = __float_as_uint(__fmaf_rn(lo2(v), inv, kRoundMagic));
+          f[2 * i + 1] = __float_as_uint(__fmaf_rn(hi2(v), inv, kRoundMagic));
+        }
+        uint32_t w[C::BITS];
+        packb<C::BITS>(f, w);
+#pragma unroll
+        for (int k = 0; k < C::BITS; ++k) qw[((g * GP) / 16 + r) * C::BITS + k] = w[k];
+      }
+      continue;
+    }
 #pragma unroll
     for (int w = 0; w < GP / 4; ++w) {
       uint32_t f[8];
@@ -558,6 +607,19 @@ __device__ __forceinline__ void dequantize(const uint32_t (&qw)[C::NQ],
   for (int g = 0; g < Gr::NL; ++g) {
     const float sk = sc[g] * C::KAPPA_INV;
     const f2 sk2 = mk2(sk, sk);
+    if constexpr (C::BITS != 4) {
+#pragma unroll
+      for (int r = 0; r < GP / 16; ++r) {
+        uint32_t w[C::BITS];
+#pragma unroll
+        for (int k = 0; k < C::BITS; ++k) w[k] = qw[((g * GP) / 16 + r) * C::BITS + k];
+        float q[32];
+        unpackb<C::BITS>(w, q);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Y[g * GP + 16 * r + i] = mul2(mk2(q[2 * i], q[2 * i + 1]), sk2);
+      }
+      continue;
+    }
 #pragma unroll
     for (int w = 0; w < GP / 4; ++w) {
       f2 q[4];
@@ -705,13 +767,14 @@ __device__ __noinline__ void drain_and_fail(uint32_t bars, const Ring& r, unsign
   atomicOr(status, 1u);
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false,
+          int BITS = 4>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                    const FwdArgs a, unsigned* status) {
-  using C = Cfg<D, ROT, TPV>;
+  using C = Cfg<D, ROT, TPV, BITS>;
   using Gr = Groups<C, G>;
-  constexpr int WARP_BYTES = S_IN * C::XTILE + S_OUT * C::QTILE;
+  constexpr int WARP_BYTES = S_IN * C::XTILE + S_OUT * C::QSTRIDE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
   __shared__ __align__(16) uint32_t s_mask[C::D];
@@ -783,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const int o = int((ring.consumed - 1) % S_OUT);
     if (lane == 0) bulk_wait_read<S_OUT - 1>();
     __syncwarp();
-    const uint32_t qdst = qbuf + uint32_t(o * C::QTILE);
+    const uint32_t qdst = qbuf + uint32_t(o * C::QSTRIDE);
     store_codes<C>(qdst, row, t, qw);
     const int64_t vrow = tile * C::VPW + row;
     if (vrow < a.n_vec) store_scales_global<C, G>(a.scales, vrow, t, sc);
@@ -800,14 +863,15 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int MINB, bool LAM = false,
+          int BITS = 4>
 __global__ void __launch_bounds__(kThreads, MINB)
     kvq_inv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                    const __grid_constant__ CUtensorMap tmX, const InvArgs a, unsigned* status) {
-  using C = Cfg<D, ROT, TPV>;
+  using C = Cfg<D, ROT, TPV, BITS>;
   using Gr = Groups<C, G>;
   constexpr int STILE = C::VPW * Gr::NG * 4;
-  constexpr int STAGE = C::QTILE + ((STILE + 1023) / 1024) * 1024;
+  constexpr int STAGE = C::QSTRIDE + ((STILE + 1023) / 1024) * 1024;
   constexpr int WARP_BYTES = S_IN * STAGE + S_OUT * C::XTILE;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars_sm[kWarps][S_IN];
@@ -1069,10 +1133,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
 }
 
 // Dynamic shared memory each kernel needs (plus 1 KiB alignment slack).
-template <int D, int ROT, int TPV, int S_IN, int S_OUT>
+template <int D, int ROT, int TPV, int S_IN, int S_OUT, int BITS = 4>
 constexpr int fwd_smem_bytes() {
-  using C = Cfg<D, ROT, TPV>;
-  return kWarps * (S_IN * C::XTILE + S_OUT * C::QTILE) + 1024;
+  using C = Cfg<D, ROT, TPV, BITS>;
+  return kWarps * (S_IN * C::XTILE + S_OUT * C::QSTRIDE) + 1024;
 }
 
 template <int D, int ROT, int TPV, int S_IN>
@@ -1081,11 +1145,11 @@ constexpr int decode_smem_bytes() {
   return kWarps * (S_IN * C::QTILE + 2 * C::XTILE) + 1024;
 }
 
-template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT>
+template <int D, int G, int ROT, int TPV, int S_IN, int S_OUT, int BITS = 4>
 constexpr int inv_smem_bytes() {
-  using C = Cfg<D, ROT, TPV>;
+  using C = Cfg<D, ROT, TPV, BITS>;
   constexpr int STILE = C::VPW * (D / G) * 4;
-  constexpr int STAGE = C::QTILE + ((STILE + 1023) / 1024) * 1024;
+  constexpr int STAGE = C::QSTRIDE + ((STILE + 1023) / 1024) * 1024;
   return kWarps * (S_IN * STAGE + S_OUT * C::XTILE) + 1024;
 }
 

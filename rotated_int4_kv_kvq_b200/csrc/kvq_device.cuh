@@ -386,4 +386,49 @@ __device__ __forceinline__ void unpack8(uint32_t w, f2 (&q)[4]) {
                __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + j)));
 }
 
+// 32 codes (the low BITS bits of each magic-rounded float, two's
+// complement) as BITS words of a little-endian bitstream: code i occupies
+// bits [BITS i, BITS i + BITS).
+template <int B>
+__device__ __forceinline__ void packb(const uint32_t (&f)[32], uint32_t (&w)[B]) {
+  if constexpr (B == 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k] = __byte_perm(__byte_perm(f[4 * k], f[4 * k + 1], 0x0040),
+                         __byte_perm(f[4 * k + 2], f[4 * k + 3], 0x0040), 0x5410);
+  } else {
+    constexpr uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+    for (int k = 0; k < B; ++k) w[k] = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t c = f[i] & mask;
+      const int pos = B * i, wi = pos / 32, sh = pos % 32;
+      w[wi] |= c << sh;
+      if (sh + B > 32) w[wi + 1] |= c >> (32 - sh);
+    }
+  }
+}
+
+// Inverse of packb: the 32 codes as exact floats.
+template <int B>
+__device__ __forceinline__ void unpackb(const uint32_t (&w)[B], float (&q)[32]) {
+  constexpr uint32_t mask = (1u << B) - 1u;
+  constexpr uint32_t sign = 1u << (B - 1);
+  // offset binary (c ^ sign) in the low mantissa bits of 2^23
+  constexpr float off = 8388608.0f + float(1 << (B - 1));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int pos = B * i, wi = pos / 32, sh = pos % 32;
+    uint32_t c;
+    if (sh + B > 32) {
+      c = __funnelshift_r(w[wi], w[wi + 1], sh);
+    } else {
+      c = w[wi] >> sh;
+    }
+    c = (c & mask) ^ sign;
+    q[i] = __uint_as_float(c | 0x4B000000u) - off;
+  }
+}
+
 }  // namespace kvq

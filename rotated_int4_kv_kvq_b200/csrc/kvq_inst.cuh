@@ -118,12 +118,12 @@ inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
   return int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count) * occ)));
 }
 
-template <int D, int G, int ROT, bool LAM>
+template <int D, int G, int ROT, bool LAM, int BITS = 4>
 cudaError_t fwd_run(const FwdLaunch& L) {
   using T = Tuning<D, ROT>;
   constexpr auto kern =
-      kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, T::FWD_MINB, LAM>;
-  constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES, T::S_OUT>();
+      kvq_fwd_kernel<D, G, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, T::FWD_MINB, LAM, BITS>;
+  constexpr int smem = fwd_smem_bytes<D, ROT, T::TPV, T::FWD_STAGES, T::S_OUT, BITS>();
   int occ;
   unsigned* st;
   cudaError_t e = setup<kern>(smem, &occ);
@@ -137,15 +137,24 @@ cudaError_t fwd_run(const FwdLaunch& L) {
 
 template <int D, int G, int ROT>
 cudaError_t fwd_one(const FwdLaunch& L) {
+  if (L.bits != 4) {
+    // other code widths: no lambda; rows of d*bits/8 bytes (3 bits needs d >= 128)
+    if (L.bits == 8) return fwd_run<D, G, ROT, false, 8>(L);
+    if (L.bits == 6) return fwd_run<D, G, ROT, false, 6>(L);
+    if constexpr (D >= 128) {
+      if (L.bits == 3) return fwd_run<D, G, ROT, false, 3>(L);
+    }
+    return cudaErrorInvalidValue;
+  }
   return L.lambda ? fwd_run<D, G, ROT, true>(L) : fwd_run<D, G, ROT, false>(L);
 }
 
-template <int D, int G, int ROT, bool LAM>
+template <int D, int G, int ROT, bool LAM, int BITS = 4>
 cudaError_t inv_run(const InvLaunch& L) {
   using T = Tuning<D, ROT>;
   constexpr auto kern =
-      kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB, LAM>;
-  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT>();
+      kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB, LAM, BITS>;
+  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, BITS>();
   int occ;
   unsigned* st;
   cudaError_t e = setup<kern>(smem, &occ);
@@ -160,6 +169,14 @@ cudaError_t inv_run(const InvLaunch& L) {
 
 template <int D, int G, int ROT>
 cudaError_t inv_one(const InvLaunch& L) {
+  if (L.bits != 4) {
+    if (L.bits == 8) return inv_run<D, G, ROT, false, 8>(L);
+    if (L.bits == 6) return inv_run<D, G, ROT, false, 6>(L);
+    if constexpr (D >= 128) {
+      if (L.bits == 3) return inv_run<D, G, ROT, false, 3>(L);
+    }
+    return cudaErrorInvalidValue;
+  }
   return L.lambda ? inv_run<D, G, ROT, true>(L) : inv_run<D, G, ROT, false>(L);
 }
 

@@ -19,6 +19,7 @@ struct FwdLaunch {
   const CUtensorMap* tmQ;  // packed [n_vec][d/2] u8, box {d/2, VPW}, swizzle = pitch
   const int8_t* signs;
   const float* lambda;     // per-channel factors [d] or NULL
+  int bits;                // code width (3, 4, 6, 8); tmQ row pitch d*bits/8
   float* scales;
   int64_t n_vec;
   int sm_count;
@@ -31,6 +32,7 @@ struct InvLaunch {
   const CUtensorMap* tmX;  // out, as x above
   const int8_t* signs;
   const float* lambda;     // per-channel factors [d] or NULL
+  int bits;                // code width (3, 4, 6, 8)
   int64_t n_vec;
   int sm_count;
   cudaStream_t stream;

@@ -22,13 +22,15 @@ STATUS = {
     0: "KVQ_OK", 1: "KVQ_ERR_NULL", 2: "KVQ_ERR_BAD_DIM", 3: "KVQ_ERR_BAD_GROUP",
     4: "KVQ_ERR_MISALIGNED", 5: "KVQ_ERR_BAD_ROT", 6: "KVQ_ERR_CUDA",
     7: "KVQ_ERR_BAD_SIZE", 8: "KVQ_ERR_DEVICE_TIMEOUT", 9: "KVQ_ERR_UNSUPPORTED_DEVICE",
+    10: "KVQ_ERR_BAD_BITS",
 }
 
 LIB_PATH = os.environ.get("KVQ_LIBRARY") or os.path.join(
     os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
 EXPORTS = ("kvq_rot_quant_fwd", "kvq_dequant_rot_inv", "kvq_rot_quant_fwd_lambda",
-           "kvq_dequant_rot_inv_lambda", "kvq_decode_step", "kvq_decode_step_windowed",
+           "kvq_dequant_rot_inv_lambda", "kvq_rot_quant_fwd_bits", "kvq_dequant_rot_inv_bits",
+           "kvq_decode_step", "kvq_decode_step_windowed",
            "kvq_attend_decode", "kvq_status_string", "kvq_device_status", "kvq_version")
 
 
@@ -57,6 +59,10 @@ def _load() -> ctypes.CDLL:
     lib.kvq_decode_step.restype = i32
     lib.kvq_decode_step_windowed.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, i32, p, i32, p]
     lib.kvq_decode_step_windowed.restype = i32
+    lib.kvq_rot_quant_fwd_bits.argtypes = [p, i64, i32, i32, i32, p, i32, p, p, p]
+    lib.kvq_rot_quant_fwd_bits.restype = i32
+    lib.kvq_dequant_rot_inv_bits.argtypes = [p, p, i64, i32, i32, i32, p, i32, p, p]
+    lib.kvq_dequant_rot_inv_bits.restype = i32
     lib.kvq_attend_decode.argtypes = [p, p, p, p, p, i64, i32, i64, i64, i32, i32, p, i32,
                                       ctypes.c_float, p, p]
     lib.kvq_attend_decode.restype = i32
@@ -155,6 +161,45 @@ def kvq_dequant_rot_inv(packed: torch.Tensor, scales: torch.Tensor, signs: torch
                                             _ptr(signs), _ptr(lam), rot, _ptr(out),
                                             _stream(stream))
         _raise("kvq_dequant_rot_inv_lambda", st)
+    return out
+
+
+def kvq_rot_quant_fwd_bits(x: torch.Tensor, signs: torch.Tensor, rot: int, group: int,
+                           bits: int, packed: torch.Tensor | None = None,
+                           scales: torch.Tensor | None = None, stream=None):
+    """Forward step with b-bit codes: packed [n_vec, d*bits/8] u8 (little-endian
+    bitstream per vector), scales [n_vec, d/group] f32."""
+    n, d = x.shape
+    qp = d * bits // 8
+    _check(x, "x", torch.float16, (n, d))
+    _check(signs, "signs", torch.int8, (d,))
+    if packed is None:
+        packed = torch.empty((n, qp), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, d // group), dtype=torch.float32, device=x.device)
+    _check(packed, "packed", torch.uint8, (n, qp))
+    _check(scales, "scales", torch.float32, (n, d // group))
+    st = lib.kvq_rot_quant_fwd_bits(_ptr(x), n, d, group, bits, _ptr(signs), rot, _ptr(packed),
+                                    _ptr(scales), _stream(stream))
+    _raise("kvq_rot_quant_fwd_bits", st)
+    return packed, scales
+
+
+def kvq_dequant_rot_inv_bits(packed: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor,
+                             rot: int, group: int, bits: int, out: torch.Tensor | None = None,
+                             stream=None):
+    """Inverse step of kvq_rot_quant_fwd_bits -> out [n_vec, d] fp16."""
+    n, qp = packed.shape
+    d = qp * 8 // bits
+    _check(packed, "packed", torch.uint8, (n, qp))
+    _check(scales, "scales", torch.float32, (n, d // group))
+    _check(signs, "signs", torch.int8, (d,))
+    if out is None:
+        out = torch.empty((n, d), dtype=torch.float16, device=packed.device)
+    _check(out, "out", torch.float16, (n, d))
+    st = lib.kvq_dequant_rot_inv_bits(_ptr(packed), _ptr(scales), n, d, group, bits, _ptr(signs),
+                                      rot, _ptr(out), _stream(stream))
+    _raise("kvq_dequant_rot_inv_bits", st)
     return out
 
 

@@ -45,17 +45,18 @@ def _sat(v):
 
 
 def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP_FRACTION,
-              lam=None):
+              lam=None, bits=4):
     """Return (codes, scales, flips, max scale rel err, flipped-row mask).
 
     `max_flip_fraction` bounds near-tie flips on realistic data; structured
     inputs (e.g. +-c vectors, whose rotations hit exact ties) pass None.
-    `lam`: per-channel factor of the lambda entry points."""
+    `lam`: per-channel factor of the lambda entry points; `bits`: code width."""
     x16 = np.asarray(x16, dtype=np.float16)
     y = O.rotated_values(x16, signs, rot, lam)
-    q_ref, s_ref = O.quantize_groups(y, group)
+    q_ref, s_ref = O.quantize_groups(y, group, bits)
     s = np.asarray(scales, dtype=np.float32)
-    q = O.unpack_nibbles(np.asarray(packed, dtype=np.uint8))
+    pk = np.asarray(packed, dtype=np.uint8)
+    q = O.unpack_nibbles(pk) if bits == 4 else O.unpack_codes(pk, bits)
     assert q.shape == q_ref.shape and s.shape == s_ref.shape
 
     # scales
@@ -66,7 +67,8 @@ def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP
     assert max_rel <= SCALE_RTOL, f"scale rel err {max_rel:.3g}"
 
     # codes
-    assert q.min(initial=0) >= -8 and q.max(initial=0) <= 7
+    qmax = 2 ** (bits - 1) - 1
+    assert q.min(initial=0) >= -qmax - 1 and q.max(initial=0) <= qmax
     diff = q.astype(np.int16) - q_ref.astype(np.int16)
     bad = diff != 0
     flips = int(bad.sum())
@@ -80,7 +82,7 @@ def check_fwd(x16, signs, rot, group, packed, scales, max_flip_fraction=MAX_FLIP
     return q, s, flips, max_rel, bad.any(axis=1)
 
 
-def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None, lam=None):
+def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None, lam=None, bits=4):
     """x_hat of the GPU against the oracle inverse of the same codes/scales,
     and against the oracle's own x_hat on rows without a code flip.  With
     `lam` the tolerance follows the channel scaling: the error of lam * x_hat
@@ -92,15 +94,15 @@ def check_inv(x16, signs, rot, group, packed, scales, out, flipped_rows=None, la
         tol = XHAT_ATOL_REL * np.maximum(np.abs(x * lam64).max(axis=1, keepdims=True),
                                          1e-30) / lam64 + np.float64(2.0 ** -24)
     with np.errstate(over="ignore"):
-        ref = _sat(O.dequant_rot_inv(packed, scales, signs, rot, group, lam))
+        ref = _sat(O.dequant_rot_inv(packed, scales, signs, rot, group, lam, bits))
     got = _sat(np.asarray(out, dtype=np.float16))
     err = np.abs(got - ref)
     inv_err = float((err / tol).max(initial=0.0))
     assert np.all(err <= tol), f"inverse error {inv_err:.3g} x tolerance"
     e2e = 0.0
-    p_ref, s_ref = O.rot_quant_fwd(np.asarray(x16, np.float16), signs, rot, group, lam)
+    p_ref, s_ref = O.rot_quant_fwd(np.asarray(x16, np.float16), signs, rot, group, lam, bits)
     with np.errstate(over="ignore"):
-        full = _sat(O.dequant_rot_inv(p_ref, s_ref, signs, rot, group, lam))
+        full = _sat(O.dequant_rot_inv(p_ref, s_ref, signs, rot, group, lam, bits))
     rows = np.ones(x.shape[0], bool) if flipped_rows is None else ~flipped_rows
     if rows.any():
         e = np.abs(got[rows] - full[rows]) / tol[rows]

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(kvq):
 
 
 def test_status_strings(kvq):
-    for code in range(10):
+    for code in range(11):
         assert kvq.status_string(code)
     assert kvq.status_string(0) == "ok"
     assert kvq.status_string(12345) == "unknown status"
@@ -148,3 +148,16 @@ def test_attend_host_checks(kvq):
     assert att(A + 8, A, A, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 4
     assert att(A, A, A + 2, A, A, 2, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 4
     assert att(A, A, A, A, A, 0, 4, 16, 10, 64, 32, A, 0, 0.125, A, None) == 0
+
+
+def test_bits_host_checks(kvq):
+    lib = kvq.lib
+    fwd, inv = lib.kvq_rot_quant_fwd_bits, lib.kvq_dequant_rot_inv_bits
+    # (x, n, d, g, bits, signs, rot, packed, scales, stream)
+    for bits in (0, 1, 2, 5, 7, 9, 16):
+        assert fwd(A, 10, 128, 32, bits, A, 0, A, A, None) == 10
+        assert inv(A, A, 10, 128, 32, bits, A, 0, A, None) == 10
+    assert fwd(A, 10, 64, 32, 3, A, 0, A, A, None) == 10  # 24-byte rows
+    assert fwd(A, 10, 96, 32, 8, A, 0, A, A, None) == 2
+    assert fwd(A, 0, 128, 32, 3, A, 0, A, A, None) == 0
+    assert inv(A, A, 0, 64, 64, 6, A, 1, A, None) == 0

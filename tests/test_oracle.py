@@ -325,6 +325,39 @@ def check_attention(rot=O.SRFT, d=64, group=32):
             np.abs(got[i].astype(np.float64) - o_).max() <= 2.0 ** -10 * np.abs(o_).max()
 
 
+def check_bitstream_golden():
+    """Little-endian bitstream, written out by hand from the two's complement
+    codes (R16): b = 3 codes 1,-1,3,-4,0,2,-2,1 are 001 111 011 100 000 010
+    110 001 LSB-first -> bytes F9 08 39; b = 6 codes 5,-20,31,-32 are 000101
+    101100 011111 100000 -> bytes 05 FB 81."""
+    q3 = np.array([[1, -1, 3, -4, 0, 2, -2, 1]], np.int8)
+    assert O.pack_codes(q3, 3).tolist() == [[0xF9, 0x08, 0x39]]
+    q6 = np.array([[5, -20, 31, -32]], np.int8)
+    assert O.pack_codes(q6, 6).tolist() == [[0x05, 0xFB, 0x81]]
+    for q, b in ((q3, 3), (q6, 6)):
+        assert np.array_equal(O.unpack_codes(O.pack_codes(q, b), b), q)
+    rng = np.random.default_rng(3)
+    q4 = rng.integers(-8, 8, (4, 64)).astype(np.int8)
+    assert np.array_equal(O.pack_codes(q4, 4), O.pack_nibbles(q4))  # b = 4 is R6
+
+
+def check_bits_quantizer(bits, d=64, group=32):
+    """b-bit groups: s = fl32(max/qmax), |q| <= qmax with qmax reached in
+    every non-zero group, error <= s/2 ([P4]), exact pack round trip."""
+    qmax = 2 ** (bits - 1) - 1
+    rng = np.random.default_rng(bits)
+    y = rng.standard_normal((50, d)) * rng.uniform(0.1, 10, (50, 1))
+    q, s = O.quantize_groups(y, group, bits)
+    yg = np.asarray(y, np.float64).astype(np.float32).reshape(50, d // group, group)
+    m = np.abs(yg).max(axis=2)
+    assert np.array_equal(s, (m / np.float32(qmax)).astype(np.float32))
+    qg = q.reshape(50, d // group, group).astype(np.int32)
+    assert np.abs(qg).max() <= qmax and np.all(np.abs(qg).max(axis=2) == qmax)
+    err = np.abs(qg * s[..., None].astype(np.float64) - yg.astype(np.float64))
+    assert np.all(err <= s[..., None].astype(np.float64) * (0.5 + 1e-6))
+    assert np.array_equal(O.unpack_codes(O.pack_codes(q, bits), bits), q)
+
+
 # ------------------------------------------------------------------ tests ---
 
 @pytest.mark.parametrize("d", [2, 4, 8, 64, 128, 256])
@@ -421,6 +454,28 @@ def test_attention(rot, d, group):
     check_attention(rot, d, group)
 
 
+def test_bitstream_golden():
+    check_bitstream_golden()
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6, 8])
+def test_bits_quantizer(bits):
+    check_bits_quantizer(bits)
+
+
+def test_bits_mse_falls_with_width():
+    """More bits, smaller error ([P1]: 6 and 8 bits are lossless in the
+    pages' test; 3 bits is worse than 4)."""
+    x = W.make_kv(W.scaled(W.config(5, d=64, group=64), heads=1, tokens=256)).numpy()
+    signs = W.make_signs(64)
+    mse = []
+    for b in (3, 4, 6, 8):
+        p, s = O.rot_quant_fwd(x, signs, O.SRFT, 64, bits=b)
+        xh = O.dequant_rot_inv(p, s, signs, O.SRFT, 64, bits=b).astype(np.float64)
+        mse.append(((xh - x.astype(np.float64)) ** 2).mean())
+    assert mse[0] > mse[1] > mse[2] > mse[3]
+
+
 def test_granularity_monotone():
     """Per-group error falls as groups shrink ("Quantization & Serving")."""
     for d in (64, 128):
@@ -496,7 +551,7 @@ def _mut_srht_bitreversed(d):
     return h[perm]
 
 
-def _mut_quant_half_away(y, group):
+def _mut_quant_half_away(y, group, bits=4):
     y32 = np.asarray(y, np.float64).astype(np.float32)
     n, d = y32.shape
     yg = y32.reshape(n, d // group, group)
@@ -507,7 +562,7 @@ def _mut_quant_half_away(y, group):
     return q.astype(np.int8).reshape(n, d), s
 
 
-def _mut_quant_div8(y, group):
+def _mut_quant_div8(y, group, bits=4):
     y32 = np.asarray(y, np.float64).astype(np.float32)
     n, d = y32.shape
     yg = y32.reshape(n, d // group, group)
@@ -563,6 +618,15 @@ def _mut_attn_fp16_keys(packed, scales, signs, rot, group):
     return x.astype(np.float16).astype(np.float64) * (1 + 2.0 ** -9)
 
 
+def _mut_pack_msb_first(q, bits):
+    q = np.asarray(q)
+    n, d = q.shape
+    u = (q.astype(np.int32) & ((1 << bits) - 1)).astype(np.uint32)
+    bitpos = np.arange(bits, dtype=np.uint32)
+    stream = ((u[..., None] >> bitpos) & 1).astype(np.uint8).reshape(n, d * bits)
+    return np.packbits(stream, axis=1, bitorder="big")
+
+
 def _mut_inverse_no_transpose(y, rot):
     return np.asarray(y, np.float64) @ O.rotation_matrix(y.shape[-1], rot).T
 
@@ -592,6 +656,7 @@ MUTATIONS = [
      [lambda: check_decode_windowed(window=4)]),
     ("rotated_values", _mut_lambda_after_rotation, [check_lambda]),
     ("dequant_rotated_f64", _mut_attn_fp16_keys, [check_attention]),
+    ("pack_codes", _mut_pack_msb_first, [check_bitstream_golden]),
 ]
 
 
