@@ -32,6 +32,12 @@ static __device__ unsigned g_status;
 #ifndef KVQ_SOUT_BIG
 #define KVQ_SOUT_BIG 1
 #endif
+#ifndef KVQ_ATTN_MAX_CLUSTER
+#define KVQ_ATTN_MAX_CLUSTER 16
+#endif
+#ifndef KVQ_ATTN_ROWS_PER_WARP
+#define KVQ_ATTN_ROWS_PER_WARP 16
+#endif
 #ifndef KVQ_FWD_MINB_64
 #define KVQ_FWD_MINB_64 5
 #endif
@@ -270,7 +276,7 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       // clusters of up to 16 blocks where the device can co-schedule them
-      int c = 8;
+      int c = std::min(8, KVQ_ATTN_MAX_CLUSTER);
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
         cudaLaunchConfig_t q = {};
@@ -279,16 +285,16 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
         q.dynamicSmemBytes = smem;
         int best = 0;
         if (cudaOccupancyMaxPotentialClusterSize(&best, kern, &q) == cudaSuccess && best >= 8)
-          c = std::min(best, 16);
+          c = std::min(std::min(best, 16), KVQ_ATTN_MAX_CLUSTER);
       }
       cudaGetLastError();
       maxc[dev] = c;
     }
     max_cluster = maxc[dev];
   }
-  // blocks per KV head (one cluster): about one staged chunk per warp, and no
-  // more than the SMs left per head (one resident block per SM)
-  constexpr int64_t per_block = int64_t(kAttnWarps) * kAttnChunk;
+  // blocks per KV head (one cluster): about KVQ_ATTN_ROWS_PER_WARP rows per
+  // warp, and no more than the SMs left per head (one resident block per SM)
+  constexpr int64_t per_block = int64_t(kAttnWarps) * KVQ_ATTN_ROWS_PER_WARP;
   const int64_t by_len = (L.len + per_block - 1) / per_block;
   const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
   const int cl = int(std::max<int64_t>(
@@ -306,7 +312,7 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cl > 1 ? 1 : 0;  // a one-block cluster needs no cluster launch
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
