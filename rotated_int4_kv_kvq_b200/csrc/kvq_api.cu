@@ -103,14 +103,20 @@ bool map_x(CUtensorMap* m, const void* base, int d, uint64_t rows, uint64_t pitc
 }
 
 // packed-code rows [rows][d/2] with row pitch `pitch` bytes, box {d/2, VPW}.
-// codes of other widths: rows of d*bits/8 bytes, box {d*bits/8, VPW}, no swizzle.
+// codes of other widths: rows of d*bits/8 bytes, moved as slabs of 128, 64
+// or 32 bytes with the matching swizzle (one unswizzled box for 48-byte rows);
+// must agree with Cfg::SW in kvq_codec.cuh.
 bool map_qb(CUtensorMap* m, const void* base, int d, int bits, uint64_t rows) {
   const uint64_t qp = uint64_t(d) * uint64_t(bits) / 8;
+  const uint32_t sw = qp % 128 == 0 ? 128 : (qp % 64 == 0 ? 64 : (qp % 32 == 0 ? 32 : 0));
+  const CUtensorMapSwizzle mode = sw == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : sw == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : sw == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                             : CU_TENSOR_MAP_SWIZZLE_NONE;
   const uint64_t dims[2] = {qp, rows};
   const uint64_t strides[1] = {qp};
-  const uint32_t box[2] = {uint32_t(qp), uint32_t(vpw_of(d))};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
+  const uint32_t box[2] = {sw ? sw : uint32_t(qp), uint32_t(vpw_of(d))};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, mode);
 }
 
 bool map_q(CUtensorMap* m, const void* base, int d, uint64_t rows, uint64_t pitch) {

@@ -61,6 +61,14 @@ struct Cfg {
   static constexpr int SLAB = VPW * 128;   // one 64-column fp16 slab
   static constexpr int QP = D * BITS / 8;  // code row pitch in bytes
   static constexpr int QMAX = (1 << (BITS - 1)) - 1;
+  // Code tiles of other widths move as NSLAB swizzled slabs of SW bytes per
+  // row (SW = 128, 64 or 32 dividing the row; 0: one unswizzled box of QP),
+  // so that rows starting on the same bank do not collide.  4-bit tiles are
+  // one box of QP bytes swizzled by their own pitch.
+  static constexpr int SW = BITS == 4 ? QP
+                            : (QP % 128 == 0 ? 128 : (QP % 64 == 0 ? 64 : (QP % 32 == 0 ? 32 : 0)));
+  static constexpr int NSLAB = SW ? QP / SW : 1;
+  static constexpr int QSLAB = VPW * (SW ? SW : QP);  // bytes of one slab
   static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
   // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
   // takes Yin = KAPPA_INV * y_hat.  SRFT (Y = packed rfft with X_0, X_{d/2}
@@ -221,6 +229,18 @@ __device__ __forceinline__ uint32_t run_byte(int t, int run) {
   return uint32_t(global_y<C>(t, 32 * run) * C::BITS / 8);
 }
 
+// Shared address of byte `o` (a multiple of 4) of `row` in a code tile of
+// another width.
+template <class C>
+__device__ __forceinline__ uint32_t code_word(uint32_t tile, int row, uint32_t o) {
+  if constexpr (C::SW == 0) {
+    return tile + uint32_t(row * C::QP) + o;
+  } else {
+    const uint32_t s = o / C::SW, b = o % C::SW;
+    return tile + s * uint32_t(C::QSLAB) + swq<C::SW>(row, int(b / 16)) + (b % 16);
+  }
+}
+
 template <class C>
 __device__ __forceinline__ void load_codes(uint32_t tile, int row, int t, uint32_t (&qw)[C::NQ]) {
   if constexpr (C::BITS == 4) {
@@ -237,7 +257,7 @@ __device__ __forceinline__ void load_codes(uint32_t tile, int row, int t, uint32
     for (int r = 0; r < C::E / 32; ++r)
 #pragma unroll
       for (int k = 0; k < C::BITS; ++k)
-        qw[r * C::BITS + k] = lds32(tile + uint32_t(row * C::QP) + run_byte<C>(t, r) + 4u * k);
+        qw[r * C::BITS + k] = lds32(code_word<C>(tile, row, run_byte<C>(t, r) + 4u * k));
   }
 }
 
@@ -254,7 +274,7 @@ __device__ __forceinline__ void store_codes(uint32_t tile, int row, int t,
     for (int r = 0; r < C::E / 32; ++r)
 #pragma unroll
       for (int k = 0; k < C::BITS; ++k)
-        sts32(tile + uint32_t(row * C::QP) + run_byte<C>(t, r) + 4u * k, qw[r * C::BITS + k]);
+        sts32(code_word<C>(tile, row, run_byte<C>(t, r) + 4u * k), qw[r * C::BITS + k]);
   }
 }
 
@@ -853,7 +873,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(&tmQ, qdst, 0, int(tile * C::VPW));
+#pragma unroll
+      for (int sl = 0; sl < C::NSLAB; ++sl)
+        tma_store_2d(&tmQ, qdst + uint32_t(sl * C::QSLAB), sl * C::SW, int(tile * C::VPW));
       bulk_commit();
     }
   }
@@ -909,7 +931,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const uint32_t bar = bars + 8u * s;
     const uint32_t dst = ibuf + uint32_t(s * STAGE);
     mbar_arrive_expect_tx(bar, C::QTILE + STILE);
-    tma_load_2d(dst, &tmQ, bar, 0, int(tile * C::VPW));
+#pragma unroll
+    for (int sl = 0; sl < C::NSLAB; ++sl)
+      tma_load_2d(dst + uint32_t(sl * C::QSLAB), &tmQ, bar, sl * C::SW, int(tile * C::VPW));
     tma_load_1d(dst + C::QTILE, &tmS, bar, int(tile * C::VPW * Gr::NG));
     ++ring.issued;
   };
