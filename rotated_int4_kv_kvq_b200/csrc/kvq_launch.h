@@ -40,7 +40,10 @@ struct InvLaunch {
 
 // Decode calls with at most this many rows (new tokens + cached rows) run
 // the one-warp-per-vector kernel (latency); larger ones the tiled kernel.
-constexpr int64_t kWideMaxRows = int64_t(1) << 16;
+#ifndef KVQ_WIDE_MAX_ROWS
+#define KVQ_WIDE_MAX_ROWS (int64_t(1) << 16)
+#endif
+constexpr int64_t kWideMaxRows = KVQ_WIDE_MAX_ROWS;
 
 struct DecodeWideLaunch {
   const uint16_t* x_new;

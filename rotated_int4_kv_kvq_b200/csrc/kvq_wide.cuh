@@ -436,25 +436,43 @@ __device__ __forceinline__ void wide_dequant_row(uint32_t code, float s, uint16_
 template <int D, int G, int ROT>
 __global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const DecodeWideArgs a) {
   constexpr int NG = D / G;
+  constexpr int GL = G / Wide<D, ROT>::W;  // lanes (chunks) per group
   const int lane = threadIdx.x & 31;
   WideLane<D, ROT> L;
   L.init(a.signs, lane);
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int64_t total = a.n_heads * (a.pos + 1);
-  for (int64_t it = gw; it < total; it += nw) {
+  // item -> (head, row): the new token of every head first, then cached rows
+  auto where = [&](int64_t it, int64_t& head, int64_t& row) {
     const bool fresh = it < a.n_heads;
-    const int64_t head = fresh ? it : (it - a.n_heads) / a.pos;
-    const int64_t row = fresh ? a.pos : (it - a.n_heads) % a.pos;
-    uint8_t* qrow = a.packed + (head * a.cap + row) * (D / 2);
-    float* srow = a.scales + (head * a.cap + row) * NG;
-    uint32_t code;  // this lane's W codes
-    float s;        // scale of this lane's group
+    head = fresh ? it : (it - a.n_heads) / a.pos;
+    row = fresh ? a.pos : (it - a.n_heads) % a.pos;
+    return fresh;
+  };
+  // the codes and scale of a cached row are loaded one item ahead, so their
+  // latency overlaps the previous row's transform
+  uint32_t code_next = 0;
+  float s_next = 0.0f;
+  auto prefetch = [&](int64_t it) {
+    int64_t head, row;
+    if (it < total && !where(it, head, row)) {
+      const int64_t r = head * a.cap + row;
+      code_next = wide_load_code<D, ROT>(a.packed + r * (D / 2), L);
+      s_next = __ldg(a.scales + r * NG + L.k2 / GL);
+    }
+  };
+  prefetch(gw);
+  for (int64_t it = gw; it < total; it += nw) {
+    int64_t head, row;
+    const bool fresh = where(it, head, row);
+    uint32_t code = code_next;  // this lane's W codes
+    float s = s_next;           // scale of this lane's group
+    prefetch(it + nw);
     if (fresh) {
+      uint8_t* qrow = a.packed + (head * a.cap + row) * (D / 2);
+      float* srow = a.scales + (head * a.cap + row) * NG;
       wide_quantize_row<D, G, ROT>(a.x_new + head * D, qrow, srow, L, code, s);
-    } else {
-      code = wide_load_code<D, ROT>(qrow, L);
-      s = __ldg(srow + L.k2 / (G / Wide<D, ROT>::W));
     }
     wide_dequant_row<D, ROT>(code, s, a.out + (head * (a.pos + 1) + row) * D, L);
   }
