@@ -47,9 +47,13 @@ FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "rotated_int4_kv_kvq_b200", "csrc")
 
 
+# the sources the tiled forward / inverse kernels are built and launched from
+CODEC_SOURCES = ("kvq_api.cu", "kvq_codec.cuh", "kvq_device.cuh", "kvq_inst.cuh", "kvq_rfft.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in CODEC_SOURCES:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
