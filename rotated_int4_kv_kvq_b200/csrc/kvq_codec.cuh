@@ -288,13 +288,36 @@ __device__ __forceinline__ constexpr float lane_sign() {
   return ((NEG >> J) & 1u) ? -1.0f : 1.0f;
 }
 
+// W_N^K (x + i y) = m (hr + i hi) in the tangent form: with c = cos, s =
+// sin of 2 pi K / N and K <= N / 8, m = c and (hr, hi) = (x + t y, y - t x),
+// t = s / c; above, m = s and t = c / s.  The caller folds m into the adds
+// that follow (fused multiply-adds), so a twiddle costs two operations
+// instead of four.
+template <int K, int N>
+__device__ __forceinline__ void twiddle_tan(float x, float y, float& m, float& hr, float& hi) {
+  if constexpr (8 * K <= N) {
+    constexpr float t = float(cos_sin_2pi(K, N).s / cos_sin_2pi(K, N).c);
+    m = tw_cos(K, N);
+    hr = fmaf(t, y, x);
+    hi = fmaf(-t, x, y);
+  } else {
+    constexpr float t = float(cos_sin_2pi(K, N).c / cos_sin_2pi(K, N).s);
+    m = tw_sin(K, N);
+    hr = fmaf(t, x, y);
+    hi = fmaf(t, y, -x);
+  }
+}
+
 // In-thread radix-2 join.  y2 is RFFT2<N/2>::fwd of the words of an N-point
 // real sequence, i.e. the packed spectra E (lane x: even samples) and O
 // (lane y: odd samples); Y receives the packed N-point rfft in the codelet
 // packing: Y[0] = (X_0, X_{N/2}) / sqrt2, Y[N/4] = X_{N/4}, and
 // X_k = E_k + W_N^k O_k, X_{N/2-k} = conj(E_k - W_N^k O_k) in Y[k],
 // Y[N/2-k].
-template <int N>
+// TAN selects the tangent-form twiddle (twiddle_tan); the plain form
+// (FMUL + FFMA per product, then the adds) measured faster in the d = 128
+// kernel only.
+template <int N, bool TAN = true>
 __device__ __forceinline__ void join_lanes_fwd(const f2 (&y2)[N / 2], f2 (&Y)[N / 2]) {
   constexpr uint64_t NEG = RFFT2<N / 2>::FWD_NEG;
   {
@@ -308,10 +331,17 @@ __device__ __forceinline__ void join_lanes_fwd(const f2 (&y2)[N / 2], f2 (&Y)[N 
     constexpr float sr = lane_sign<NEG, 2 * k>(), si = lane_sign<NEG, 2 * k + 1>();
     const float er = sr * lo2(y2[2 * k]), orr = sr * hi2(y2[2 * k]);
     const float ei = si * lo2(y2[2 * k + 1]), oi = si * hi2(y2[2 * k + 1]);
-    constexpr float c = tw_cos(k, N), s = tw_sin(k, N);
-    const float gr = fmaf(c, orr, s * oi), gi = fmaf(c, oi, -(s * orr));  // W_N^k O_k
-    Y[k] = mk2(er + gr, ei + gi);
-    Y[N / 2 - k] = mk2(er - gr, gi - ei);
+    if constexpr (TAN) {
+      float m, hr, hi;  // W_N^k O_k = m (hr, hi)
+      twiddle_tan<k, N>(orr, oi, m, hr, hi);
+      Y[k] = mk2(fmaf(m, hr, er), fmaf(m, hi, ei));
+      Y[N / 2 - k] = mk2(fmaf(-m, hr, er), fmaf(m, hi, -ei));
+    } else {
+      constexpr float c = tw_cos(k, N), s = tw_sin(k, N);
+      const float gr = fmaf(c, orr, s * oi), gi = fmaf(c, oi, -(s * orr));  // W_N^k O_k
+      Y[k] = mk2(er + gr, ei + gi);
+      Y[N / 2 - k] = mk2(er - gr, gi - ei);
+    }
   });
 }
 
@@ -344,11 +374,11 @@ __device__ __forceinline__ void pair_join_fwd(const f2 (&y)[C::D / 4], int t, f2
     // thread 0 twiddles conj(received) = O_a, thread 1 its own V_a
     const float tx = odd ? ox : rx, ty = odd ? oy : -ry;
     const float px = odd ? rx : ox, py = odd ? -ry : oy;  // E (thread 1: conj E)
-    constexpr float c = tw_cos(a, C::D), s = tw_sin(a, C::D);
-    const float gx = fmaf(c, tx, s * ty), gy = fmaf(c, ty, -(s * tx));  // W_d^a t
-    const float qx = odd ? gy : gx, qy = odd ? -gx : gy;
-    if constexpr (a < H / 2) Y[a] = mk2(px + qx, py + qy);
-    Y[H - a] = mk2(px - qx, qy - py);
+    float m, hx, hy;  // W_d^a t = m (hx, hy)
+    twiddle_tan<a, C::D>(tx, ty, m, hx, hy);
+    const float qx = odd ? hy : hx, qy = odd ? -hx : hy;  // q / m
+    if constexpr (a < H / 2) Y[a] = mk2(fmaf(m, qx, px), fmaf(m, qy, py));
+    Y[H - a] = mk2(fmaf(-m, qx, px), fmaf(m, qy, -py));
   });
 }
 
@@ -386,7 +416,7 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
     }
     RFFT2<C::E / 2>::fwd(u, y2);
     if constexpr (C::TPV == 1) {
-      join_lanes_fwd<C::E>(y2, Y);
+      join_lanes_fwd<C::E, C::D != 128>(y2, Y);
     } else {
       f2 yt[C::P];
       join_lanes_fwd<C::E>(y2, yt);
