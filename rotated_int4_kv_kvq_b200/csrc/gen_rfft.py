@@ -134,11 +134,19 @@ class Graph:
         if 4 * k == 3 * n:
             return self.mul_mi(a) if sign > 0 else self.mul_i(a)
         ang = 2.0 * math.pi * k / n
-        c = float(np.float32(math.cos(ang)))
-        s = float(np.float32(sign * math.sin(ang)))
-        # (ar + i ai)(c + i s) = (ar c - ai s) + i (ar s + ai c)
-        re = self.fmac(a[0], c, self.mulc(a[1], -s))
-        im = self.fmac(a[0], s, self.mulc(a[1], c))
+        cd, sd = math.cos(ang), sign * math.sin(ang)
+        # Tangent form: (ar + i ai)(c + i s) = c [(ar - t ai) + i (ai + t ar)]
+        # with t = s / c (or s [(t ar - ai) + i (ar + t ai)], t = c / s, when
+        # |s| > |c|): one multiply-add per component, and the common factor
+        # a multiply that the emitter folds into the adds consuming it.
+        if abs(cd) >= abs(sd):
+            t, m = float(np.float32(sd / cd)), float(np.float32(cd))
+            re = self.mulc(self.fmac(a[1], -t, a[0]), m)
+            im = self.mulc(self.fmac(a[0], t, a[1]), m)
+        else:
+            t, m = float(np.float32(cd / sd)), float(np.float32(sd))
+            re = self.mulc(self.fmac(a[0], t, self.neg(a[1])), m)
+            im = self.mulc(self.fmac(a[1], t, a[0]), m)
         return (re, im)
 
 
@@ -330,26 +338,40 @@ def emit_x2(name, g: Graph, outs, in_arr, out_arr, n):
     the polarity of every output is returned for the caller to absorb.
     Returns (code, op count, output polarities, op list for `run_x2`)."""
     live = live_nodes(g, outs)
-    uses = use_counts(g, outs, live)
-    fused = {}
-    absorbed = set()
+    # A multiply by a constant whose every consumer is an add/sub disappears:
+    # each consumer becomes one multiply-add (same cost as the add).
+    users = {i: [] for i in live}
     for i in sorted(live):
         op, args = g.nodes[i]
-        if op not in ("add", "sub"):
+        if op in ("add", "sub"):
+            users[args[0]].append(i)
+            users[args[1]].append(i)
+        elif op == "mul":
+            users[args[0]].append(i)
+        elif op == "fma":
+            users[args[0]].append(i)
+            users[args[2]].append(i)
+    out_nodes = {o.node for o in outs if o.node is not None}
+    fused = {}
+    absorbed = set()
+    for m in sorted(live):
+        if g.nodes[m][0] != "mul" or m in out_nodes or not users[m]:
             continue
-        for pos in (1, 0):
-            m = args[pos]
-            mop, margs = g.nodes[m]
-            if mop == "mul" and uses[m] == 1 and m not in absorbed:
-                other = args[1 - pos]
-                if op == "add":
-                    fused[i] = (m, +1, other, +1)
-                elif pos == 1:
-                    fused[i] = (m, -1, other, +1)
-                else:
-                    fused[i] = (m, +1, other, -1)
-                absorbed.add(m)
-                break
+        us = users[m]
+        if len(set(us)) != len(us) or any(
+                g.nodes[i][0] not in ("add", "sub") or i in fused for i in us):
+            continue
+        for i in us:
+            op, args = g.nodes[i]
+            pos = 1 if args[1] == m else 0
+            other = args[1 - pos]
+            if op == "add":
+                fused[i] = (m, +1, other, +1)
+            elif pos == 1:
+                fused[i] = (m, -1, other, +1)
+            else:
+                fused[i] = (m, +1, other, -1)
+        absorbed.add(m)
     pol = {}
     prog = []  # (dst, op, a, b, const): op in add/sub/mul/fma; fma = a*const + b
     lines = [f"__device__ __forceinline__ void {name}(const f2 (&{in_arr})[{n}], "
