@@ -9,20 +9,27 @@ register):
   rfft<n>x2_fwd(x, y):  y[0] = X_0/sqrt2, y[1] = X_{n/2}/sqrt2,
                         y[2k] = Re X_k, y[2k+1] = Im X_k   (1 <= k < n/2),
                         X_k = sum_m x_m exp(-2 pi i k m / n)  (unnormalized);
-  rfft<n>x2_inv(y, x):  the transpose map, x_m = sum_k X_k exp(+2 pi i k m / n)
-                        with X rebuilt from y in the same packing (X_0 =
-                        sqrt2 y[0], X_{n/2} = sqrt2 y[1]).
+  rfft<n>x2_inv(y, x):  the transpose (adjoint) of the forward map,
+                        x_m = (1/2) sum_k X_k exp(+2 pi i k m / n) with X
+                        rebuilt from y in the same packing (X_0 = sqrt2 y[0],
+                        X_{n/2} = sqrt2 y[1]), i.e. half the unnormalized
+                        inverse real DFT.
 
-The transforms follow the split-radix decomposition for real data (even
-samples through a half-length real DFT, samples 4m+1 and 4m+3 through two
-quarter-length real DFTs, recombined with twiddles W^k and W^3k), keeping
-only the non-redundant half of every Hermitian spectrum.  The generator
-builds an expression graph with hash-consing, folds trivial twiddles
-(+-1, +-i) and negations into add/sub, writes twiddle products as fused
-multiply-adds, checks the graph numerically against numpy's FFT, then
-checks the emitted instruction list (with the polarity of every output, see
-emit_x2) against the graph before writing anything.  Twiddle constants are
-cos/sin evaluated in double and rounded once to float.
+The forward transform follows the split-radix decomposition for real data
+(even samples through a half-length real DFT, samples 4m+1 and 4m+3
+through two quarter-length real DFTs, recombined with twiddles W^k and
+W^3k), keeping only the non-redundant half of every Hermitian spectrum; the
+inverse is its transpose, built by reversing every edge of the forward
+graph, so it costs the same number of operations.  The generator builds an
+expression graph with hash-consing, folds trivial twiddles (+-1, +-i) and
+negations into add/sub, writes a twiddle product in tangent form (c (x +
+(s/c) y), or with the roles of c and s swapped) so that the common factor
+is a multiply that can be carried: a sum of two such multiples keeps one
+factor outside (one multiply-add), and a multiply whose consumers are all
+adds is folded into them.  It checks the graph numerically against numpy's
+FFT, then the emitted instruction list (with the polarity of every output,
+see emit_x2) against the graph before writing anything.  Twiddle constants
+are evaluated in double and rounded once to float.
 """
 
 from __future__ import annotations
@@ -89,6 +96,10 @@ class Graph:
             return a
         if c == -1.0:
             return self.neg(a)
+        op, args = self.nodes[a.node]
+        if op == "mul":  # (x m) c = x (m c): one multiply, not two
+            x, m = args
+            return self.mulc(R(x, a.sign), float(np.float32(m * c)))
         s = a.sign * (1 if c > 0 else -1)
         return R(self._mk("mul", a.node, abs(c)), s)
 
@@ -102,6 +113,42 @@ class Graph:
             return self.add(self.mulc(a, c), b)
         cc = a.sign * b.sign * c
         return R(self._mk("fma", a.node, cc, b.node), b.sign)
+
+    def split_mul(self, a):
+        """a = m * x with x a node: (x, m); (a, None) when a is no multiple."""
+        if a.node is None:
+            return a, None
+        op, args = self.nodes[a.node]
+        if op == "mul":
+            return R(args[0], a.sign), args[1]
+        return a, None
+
+    def add_common(self, a, b, sb=1):
+        """a + sb * b; when both are constant multiples m_a x, m_b y, as
+        m_a (x + sb (m_b / m_a) y): one multiply-add, the factor m_a left for
+        the emitter to fold into the adds that consume the sum."""
+        xa, ma = self.split_mul(a)
+        xb, mb = self.split_mul(b)
+        if ma is None or mb is None:
+            return self.add(a, b) if sb > 0 else self.sub(a, b)
+        r = float(np.float32(sb * mb / ma))
+        return self.mulc(self.fmac(xb, r, xa), ma)
+
+    def fmac_common(self, a, c, b):
+        """c a + b; a constant factor of a is folded into c, and one of b is
+        kept out (as for add_common)."""
+        xa, ma = self.split_mul(a)
+        xb, mb = self.split_mul(b)
+        ca = c if ma is None else float(np.float32(c * ma))
+        if mb is None:
+            return self.fmac(xa, ca, b)
+        return self.mulc(self.fmac(xa, float(np.float32(ca / mb)), xb), mb)
+
+    def cadd_common(self, a, b):
+        return (self.add_common(a[0], b[0]), self.add_common(a[1], b[1]))
+
+    def csub_common(self, a, b):
+        return (self.add_common(a[0], b[0], -1), self.add_common(a[1], b[1], -1))
 
     # complex helpers: values are (re, im) pairs of R
     def cadd(self, a, b):
@@ -141,26 +188,30 @@ class Graph:
         # a multiply that the emitter folds into the adds consuming it.
         if abs(cd) >= abs(sd):
             t, m = float(np.float32(sd / cd)), float(np.float32(cd))
-            re = self.mulc(self.fmac(a[1], -t, a[0]), m)
-            im = self.mulc(self.fmac(a[0], t, a[1]), m)
+            re = self.mulc(self.fmac_common(a[1], -t, a[0]), m)
+            im = self.mulc(self.fmac_common(a[0], t, a[1]), m)
         else:
             t, m = float(np.float32(cd / sd)), float(np.float32(sd))
-            re = self.mulc(self.fmac(a[0], t, self.neg(a[1])), m)
-            im = self.mulc(self.fmac(a[1], t, a[0]), m)
+            re = self.mulc(self.fmac_common(a[0], t, self.neg(a[1])), m)
+            im = self.mulc(self.fmac_common(a[1], t, a[0]), m)
         return (re, im)
 
 
-def rdft(g: Graph, x):
+def rdft(g: Graph, x, top=True):
     """Real DFT of x (list of R, len n): returns X_k as (re, im) for
-    k = 0..n/2 (X_0 and X_{n/2} real)."""
+    k = 0..n/2 (X_0 and X_{n/2} real).  Below the top level the outputs may
+    carry a constant factor (a multiply node) that the parent folds into
+    its own operations."""
     n = len(x)
     if n == 1:
         return [(x[0], ZERO)]
     if n == 2:
         return [(g.add(x[0], x[1]), ZERO), (g.sub(x[0], x[1]), ZERO)]
-    e = rdft(g, x[0::2])  # n/2: k = 0..n/4
-    u = rdft(g, x[1::4])  # n/4: k = 0..n/8
-    v = rdft(g, x[3::4])
+    e = rdft(g, x[0::2], False)  # n/2: k = 0..n/4
+    u = rdft(g, x[1::4], False)  # n/4: k = 0..n/8
+    v = rdft(g, x[3::4], False)
+    cadd = g.cadd if top else g.cadd_common
+    csub = g.csub if top else g.csub_common
 
     def full(h, m, k):  # value at k of a Hermitian spectrum of length m
         k %= m
@@ -179,12 +230,12 @@ def rdft(g: Graph, x):
         a[k] = Graph.mul_mi(Graph.conj(a[q - k]))
         b[k] = Graph.mul_i(Graph.conj(b[q - k]))
     for k in range(0, q):
-        s = g.cadd(a[k], b[k])
-        dd = g.csub(a[k], b[k])
-        out[k] = g.cadd(full(e, n // 2, k), s)
-        out[k + q] = g.cadd(full(e, n // 2, k + q), Graph.mul_mi(dd))
-    s0 = g.cadd(a[0], b[0])
-    out[n // 2] = g.csub(full(e, n // 2, 0), s0)
+        s = (g.add_common(a[k][0], b[k][0]), g.add_common(a[k][1], b[k][1]))
+        dd = (g.add_common(a[k][0], b[k][0], -1), g.add_common(a[k][1], b[k][1], -1))
+        out[k] = cadd(full(e, n // 2, k), s)
+        out[k + q] = cadd(full(e, n // 2, k + q), Graph.mul_mi(dd))
+    s0 = g.cadd_common(a[0], b[0])
+    out[n // 2] = csub(full(e, n // 2, 0), s0)
     return out
 
 
@@ -195,20 +246,20 @@ def irdft(g: Graph, xs):
     if n == 1 or len(xs) == 1:
         return [xs[0][0]]
     if n == 2:
-        return [g.add(xs[0][0], xs[1][0]), g.sub(xs[0][0], xs[1][0])]
+        return [g.add_common(xs[0][0], xs[1][0]), g.add_common(xs[0][0], xs[1][0], -1)]
 
     def full(k):
         k %= n
         return xs[k] if k <= n // 2 else Graph.conj(xs[n - k])
 
     q = n // 4
-    ep = [g.cadd(full(k), full(k + n // 2)) for k in range(0, q + 1)]
+    ep = [g.cadd_common(full(k), full(k + n // 2)) for k in range(0, q + 1)]
     up, vp = [], []
     for k in range(0, n // 8 + 1):
-        d1 = g.csub(full(k), full(k + n // 2))
-        d2 = g.csub(full(k + q), full(k + 3 * q))
-        up.append(g.ctw(g.cadd(d1, Graph.mul_i(d2)), k, n, +1))
-        vp.append(g.ctw(g.csub(d1, Graph.mul_i(d2)), 3 * k, n, +1))
+        d1 = g.csub_common(full(k), full(k + n // 2))
+        d2 = g.csub_common(full(k + q), full(k + 3 * q))
+        up.append(g.ctw(g.cadd_common(d1, Graph.mul_i(d2)), k, n, +1))
+        vp.append(g.ctw(g.csub_common(d1, Graph.mul_i(d2)), 3 * k, n, +1))
     xe = irdft(g, ep)
     xu = irdft(g, up)
     xv = irdft(g, vp)
@@ -233,14 +284,57 @@ def build_forward(n):
     return g, outs
 
 
+def transpose(g: Graph, outs, n, in_name, out_name):
+    """The adjoint of the linear map x -> outs (inputs named in_name[i]):
+    a graph from inputs out_name[j] to n outputs, each original edge
+    reversed with its coefficient (a fan-out becomes a sum).  Same number
+    of operations as the original, give or take its input/output counts."""
+    live = live_nodes(g, outs)
+    cons = {i: [] for i in live}  # node -> [(consumer, coefficient)]
+    for i in sorted(live):
+        op, args = g.nodes[i]
+        if op == "add":
+            cons[args[0]].append((i, 1.0))
+            cons[args[1]].append((i, 1.0))
+        elif op == "sub":
+            cons[args[0]].append((i, 1.0))
+            cons[args[1]].append((i, -1.0))
+        elif op == "mul":
+            cons[args[0]].append((i, args[1]))
+        elif op == "fma":
+            cons[args[0]].append((i, args[1]))
+            cons[args[2]].append((i, 1.0))
+    gt = Graph()
+    seeds = {i: [] for i in live}
+    for j, o in enumerate(outs):
+        if o.node is not None:
+            seeds[o.node].append(gt.mulc(gt.inp(f"{out_name}[{j}]"), float(o.sign)))
+    tval = {}
+    for i in sorted(live, reverse=True):  # every consumer has a larger index
+        terms = [(t, 1.0) for t in seeds[i]] + [(tval[c], w) for c, w in cons[i]]
+
+        def scaled(tw):  # a term that would start the sum with a factor
+            t, w = tw
+            return abs(w) != 1.0 or gt.split_mul(t)[1] is not None
+
+        terms.sort(key=scaled)  # an unscaled term first: no factor to carry
+        acc = ZERO
+        for t, w in terms:
+            acc = gt.fmac_common(t, w, acc) if acc.node is not None else gt.mulc(t, w)
+        tval[i] = acc
+    res = []
+    for k in range(n):
+        key = ("in", (f"{in_name}[{k}]",))
+        node = g.memo.get(key)
+        res.append(tval.get(node, ZERO) if node is not None else ZERO)
+    return gt, res
+
+
 def build_inverse(n):
-    g = Graph()
-    y = [g.inp(f"y[{i}]") for i in range(n)]
-    xs = [(g.mulc(y[0], R2), ZERO)]
-    xs += [(y[2 * k], y[2 * k + 1]) for k in range(1, n // 2)]
-    xs += [(g.mulc(y[1], R2), ZERO)]
-    outs = irdft(g, xs)
-    return g, outs
+    """The adjoint of build_forward: x = A^T y (half the unnormalized inverse
+    real DFT of the packed spectrum y)."""
+    g, outs = build_forward(n)
+    return transpose(g, outs, n, "x", "y")
 
 
 def evaluate(g: Graph, outs, inputs: dict):
@@ -302,7 +396,7 @@ def check(n):
         Xs[0] = yv[0] * math.sqrt(2)
         Xs[n // 2] = yv[1] * math.sqrt(2)
         Xs[1:n // 2] = yv[2::2][: n // 2 - 1] + 1j * yv[3::2][: n // 2 - 1]
-        ref = np.fft.irfft(Xs, n) * n
+        ref = np.fft.irfft(Xs, n) * (n / 2)
         err = np.abs(got - ref).max() / np.abs(ref).max()
         assert err < 1e-6, (n, "inverse", err)
 

@@ -73,7 +73,9 @@ struct Cfg {
   // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
   // takes Yin = KAPPA_INV * y_hat.  SRFT (Y = packed rfft with X_0, X_{d/2}
   // over sqrt2, from the generated real-FFT codelets, joined across the pair
-  // at d = 256): sqrt(2/d) and 1/sqrt(2d).  SRHT: 1/sqrt(d) both ways.
+  // at d = 256; the inverse codelet is the forward one's transpose, half the
+  // unnormalized inverse DFT): sqrt(2/d) both ways.  SRHT: 1/sqrt(d) both
+  // ways.
   static constexpr bool CODELET = ROT == kRotSRFT && TPV == 1;
   // Thread-pair SRFT: each thread runs a d/2-point real FFT on the even
   // (thread 0) or odd (thread 1) samples; one half-volume exchange joins them.
@@ -81,7 +83,7 @@ struct Cfg {
   static constexpr double KAPPA_FWD_D =
       ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : const_sqrt(2.0 / D);
   static constexpr double KAPPA_INV_D =
-      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : 1.0 / const_sqrt(2.0 * D);
+      ROT == kRotSRHT ? 1.0 / const_sqrt(double(D)) : const_sqrt(2.0 / D);
   static constexpr float KAPPA_INV = float(KAPPA_INV_D);
   static constexpr float KAPPA7 = float(KAPPA_FWD_D / QMAX);  // stored scale = m * KAPPA7
   static_assert(D % 64 == 0 && (TPV == 1 || TPV == 2), "shape");

@@ -19,8 +19,9 @@
 // X_k, k in [C k2, C k2 + C), i.e. the chunk y[W k2 .. W k2 + W) of the
 // packed spectrum.  The real split pairs Z_k with Z_{N-k}: for k1 >= 1 the
 // partner sits in lane l ^ 31, register C - k1; for k1 = 0 in lane
-// bitrev5(-k2 mod 32), register 0.  Scaling follows the half-length complex
-// path of kvq_codec.cuh (Y = 2X packing, KAPPA = 1/sqrt(2d) both ways).
+// bitrev5(-k2 mod 32), register 0.  Scaling: the unnormalized packed
+// spectrum is Y = 2X (y = KAPPA Y), and the inverse takes Yin = KAPPA y_hat,
+// KAPPA = 1/sqrt(2d) both ways.
 #pragma once
 
 #include "kvq_device.cuh"
