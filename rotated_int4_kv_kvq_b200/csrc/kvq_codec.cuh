@@ -34,13 +34,15 @@ constexpr int kThreads = kWarps * 32;
 
 // Where a thread's E local rotated coordinates sit in the vector's y:
 //  kLayFull    (one thread per vector): local i is y[i].
-//  kLayHalf    (SRHT, thread pair):     thread t holds y[t*E + i].
+//  kLayHadamard (SRHT, thread pair):    local half h (E/2 values) of thread
+//           t is quarter 2h + t of y: thread 0 holds quarters 0 and 2,
+//           thread 1 quarters 1 and 3 (see rotate_fwd).
 //  kLayQuarter (SRFT, thread pair):     local half h (E/2 values) of thread t is
 //           quarter qd = h ? 3 - 2t : 2t of y, i.e. thread 0 holds quarters
 //           0 and 3 and thread 1 quarters 2 and 1.  This is where the pair
 //           join of the two half-length real FFTs leaves each output (see
 //           pair_join_fwd); both halves are in natural y order.
-constexpr int kLayFull = 0, kLayHalf = 1, kLayQuarter = 2;
+constexpr int kLayFull = 0, kLayHadamard = 1, kLayQuarter = 2;
 
 template <int D_, int ROT_, int TPV_, int BITS_ = 4>
 struct Cfg {
@@ -69,7 +71,7 @@ struct Cfg {
                             : (QP % 128 == 0 ? 128 : (QP % 64 == 0 ? 64 : (QP % 32 == 0 ? 32 : 0)));
   static constexpr int NSLAB = SW ? QP / SW : 1;
   static constexpr int QSLAB = VPW * (SW ? SW : QP);  // bytes of one slab
-  static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHalf);
+  static constexpr int LAYOUT = TPV == 1 ? kLayFull : (ROT == kRotSRFT ? kLayQuarter : kLayHadamard);
   // y = KAPPA_FWD * Y (Y: rotate_fwd's unnormalized output) and the inverse
   // takes Yin = KAPPA_INV * y_hat.  SRFT (Y = packed rfft with X_0, X_{d/2}
   // over sqrt2, from the generated real-FFT codelets, joined across the pair
@@ -105,8 +107,8 @@ template <class C>
 __device__ __forceinline__ int global_y(int t, int i) {
   if constexpr (C::LAYOUT == kLayFull) {
     return i;
-  } else if constexpr (C::LAYOUT == kLayHalf) {
-    return t * C::E + i;
+  } else if constexpr (C::LAYOUT == kLayHadamard) {
+    return (2 * (i / (C::E / 2)) + t) * (C::D / 4) + i % (C::E / 2);
   } else {
     return quarter_of(t, i / (C::E / 2)) * (C::D / 4) + i % (C::E / 2);
   }
@@ -120,7 +122,9 @@ __device__ __forceinline__ uint32_t sign_mask_word(const int8_t* signs, int w) {
 // Sign mask of word j of thread t as load_x hands it out.  Thread-pair SRFT:
 // thread t holds v_m = u_{2m+t} (-1)^{t m}, word j = (v_{2j}, v_{2j+1}); the
 // modulation (-1)^m of thread 1 moves its spectrum by d/4 bins.  Otherwise
-// thread t holds words t*NW + j.
+// thread t holds words t*NW + j; thread-pair SRHT: thread 1's second half
+// negated (a sign pattern on the input of a Walsh-Hadamard transform is a
+// permutation of its output, see rotate_fwd).
 template <class C>
 __device__ __forceinline__ uint32_t load_mask_word(const int8_t* signs, int t, int j) {
   if constexpr (C::PAIR_RFFT) {
@@ -128,7 +132,9 @@ __device__ __forceinline__ uint32_t load_mask_word(const int8_t* signs, int t, i
     const bool hi = (signs[4 * j + 2 + t] < 0) != (t == 1);
     return (lo ? 0x00008000u : 0u) | (hi ? 0x80000000u : 0u);
   } else {
-    return sign_mask_word(signs, t * C::NW + j);
+    uint32_t m = sign_mask_word(signs, t * C::NW + j);
+    if (C::ROT == kRotSRHT && C::TPV == 2 && t == 1 && j >= C::NW / 2) m ^= 0x80008000u;
+    return m;
   }
 }
 
@@ -139,6 +145,8 @@ __device__ __forceinline__ uint32_t load_mask_word(const int8_t* signs, int t, i
 template <class C>
 __device__ __forceinline__ uint32_t store_mask_word(const int8_t* signs, int t, int j) {
   uint32_t m = sign_mask_word(signs, t * C::NW + j);
+  // thread-pair SRHT: thread 1's second half arrives negated (rotate_inv)
+  if (C::ROT == kRotSRHT && C::TPV == 2 && t == 1 && j >= C::NW / 2) m ^= 0x80008000u;
   if constexpr (C::ROT == kRotSRFT) {
     constexpr uint64_t neg = RFFT2<C::E / 2>::INV_NEG;  // inverse codelet polarity
     if constexpr (C::TPV == 1) {
@@ -400,11 +408,23 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
       if constexpr (LAM) Y[j] = mul2(Y[j], lds_f2(lam + 8u * j));
     }
     fwht<C::P>(Y);
-    if constexpr (C::TPV == 2) {  // H_d = [[H, H], [H, -H]] across the pair
-      const float sg = t ? -1.0f : 1.0f;
-      const f2 sg2 = mk2(sg, sg);
+    if constexpr (C::TPV == 2) {
+      // H_d = [[H, H], [H, -H]] across the pair, exchanging half the data.
+      // Thread 1's input carries the sign (-1)^{bit log2(E/2) of n} (its load
+      // mask), and a Walsh-Hadamard transform turns that sign pattern into
+      // the index shift k -> k ^ E/2 of its output: its first P/2 pairs hold
+      // outputs E/2..E-1, the rest 0..E/2-1.  Both threads send pairs
+      // P/2..P-1 and keep 0..P/2-1, so each holds (H x_lo)_k and (H x_hi)_k
+      // for its quarter of k (thread 0: k < E/2) and forms y_k = lo + hi,
+      // y_{k+d/2} = lo - hi; thread 1's difference is hi - lo, negated
+      // (quantize takes it back).
+      constexpr int H = C::P / 2;
 #pragma unroll
-      for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
+      for (int i = 0; i < H; ++i) {
+        const f2 own = Y[i], r = shfl_xor2(Y[H + i], 1);
+        Y[i] = add2(own, r);
+        Y[H + i] = sub2(own, r);
+      }
     }
   } else {
     // Each word is (even, odd) sample: one two-lane codelet transforms both
@@ -510,10 +530,21 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
   };
   if constexpr (C::ROT == kRotSRHT) {
     if constexpr (C::TPV == 2) {
+      // Inverse of rotate_fwd's pair step: from a = y_k, b = y_{k+d/2} of
+      // this thread's quarter of k, thread 0 keeps the sums a + b and sends
+      // the differences a - b, thread 1 the other way round; thread 0 then
+      // holds y_lo + y_hi in order, thread 1 y_lo - y_hi with its halves
+      // swapped, whose transform carries the sign (-1)^{bit log2(E/2) of m}
+      // (taken back by its store mask).
+      constexpr int H = C::P / 2;
       const float sg = t ? -1.0f : 1.0f;
-      const f2 sg2 = mk2(sg, sg);
+      const f2 sg2 = mk2(sg, sg), nsg2 = mk2(-sg, -sg);
 #pragma unroll
-      for (int i = 0; i < C::P; ++i) Y[i] = fma2(sg2, Y[i], shfl_xor2(Y[i], 1));
+      for (int i = 0; i < H; ++i) {
+        const f2 a = Y[i], b = Y[H + i];
+        Y[i] = fma2(sg2, b, a);
+        Y[H + i] = shfl_xor2(fma2(nsg2, b, a), 1);
+      }
     }
     fwht<C::P>(Y);
 #pragma unroll
@@ -551,17 +582,23 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
 
 // ------------------------------------------------------ quantize / pack ---
 
-constexpr int kXNone = 0, kXShared = 1, kXCrossHalf = 2, kXAll = 3;
+// How a group's absmax is formed: kXNone within the thread, kXCrossHalf
+// local half h of one thread with local half 1 - h of the other, kXPaired
+// local half h of both threads, kXAll the whole vector over the pair.
+constexpr int kXNone = 0, kXCrossHalf = 1, kXPaired = 2, kXAll = 3;
 
 template <class C, int G>
 struct Groups {
   static constexpr int GL =
-      C::LAYOUT == kLayQuarter ? (G <= C::E / 2 ? G : C::E / 2) : (G <= C::E ? G : C::E);
+      C::LAYOUT == kLayFull ? (G <= C::E ? G : C::E) : (G <= C::E / 2 ? G : C::E / 2);
   static constexpr int NL = C::E / GL;  // local groups (scales) per thread
   static constexpr int NG = C::D / G;   // scales per vector
-  static constexpr int X = C::LAYOUT == kLayFull    ? kXNone
-                           : C::LAYOUT == kLayHalf  ? (G > C::E ? kXShared : kXNone)
-                           : (G <= C::E / 2 ? kXNone : (G == C::D / 2 ? kXCrossHalf : kXAll));
+  static constexpr int X =
+      C::LAYOUT == kLayFull
+          ? kXNone
+          : (G <= C::E / 2 ? kXNone
+                           : (G == C::D / 2 ? (C::LAYOUT == kLayQuarter ? kXCrossHalf : kXPaired)
+                                            : kXAll));
   static_assert(GL % 16 == 0, "group");
 };
 
@@ -571,6 +608,7 @@ __device__ __forceinline__ int global_group(int t, int lg) {
   using Gr = Groups<C, G>;
   if constexpr (Gr::X == kXNone) return global_y<C>(t, lg * Gr::GL) / G;
   if constexpr (Gr::X == kXCrossHalf) return quarter_of(t, lg) / 2;
+  if constexpr (Gr::X == kXPaired) return lg;
   return 0;
 }
 
@@ -583,16 +621,20 @@ __device__ __forceinline__ bool writes_scale(int t, int lg) {
   return t == 0;
 }
 
+// Codes and scales of thread t's values Y.  Thread-pair SRHT: thread 1's
+// second local half holds -y (rotate_fwd), quantized with the sign taken
+// back.
 template <class C, int G>
 __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::NQ],
-                                         float (&sc)[Groups<C, G>::NL]) {
+                                         float (&sc)[Groups<C, G>::NL], int t) {
   using Gr = Groups<C, G>;
   constexpr int GP = Gr::GL / 2;  // pairs per local group
   float m[Gr::NL];
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) m[g] = absmax2<GP>(&Y[g * GP]);
-  if constexpr (Gr::X == kXShared) {
-    m[0] = fmaxf(m[0], __shfl_xor_sync(kFull, m[0], 1));
+  if constexpr (Gr::X == kXPaired) {
+#pragma unroll
+    for (int g = 0; g < Gr::NL; ++g) m[g] = fmaxf(m[g], __shfl_xor_sync(kFull, m[g], 1));
   } else if constexpr (Gr::X == kXCrossHalf) {
     const float o0 = __shfl_xor_sync(kFull, m[0], 1), o1 = __shfl_xor_sync(kFull, m[1], 1);
     m[0] = fmaxf(m[0], o1);
@@ -606,7 +648,10 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
   const f2 magic = mk2(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int g = 0; g < Gr::NL; ++g) {
-    const float inv = m[g] > 0.0f ? __fdiv_rn(float(C::QMAX), m[g]) : 0.0f;
+    float inv = m[g] > 0.0f ? __fdiv_rn(float(C::QMAX), m[g]) : 0.0f;
+    if constexpr (C::LAYOUT == kLayHadamard) {
+      if (t == 1 && g >= Gr::NL / 2) inv = -inv;
+    }
     sc[g] = m[g] * C::KAPPA7;
     const f2 inv2 = mk2(inv, inv);
     if constexpr (C::BITS != 4) {
@@ -766,8 +811,8 @@ __device__ __forceinline__ void store_scales_global(float* scales, int64_t vrow,
   using Gr = Groups<C, G>;
   float* row = scales + vrow * Gr::NG;
   if constexpr (Gr::X == kXNone) {
-    // runs of R consecutive scales (two runs per thread in the quarter layout)
-    constexpr int R = C::LAYOUT == kLayQuarter ? Gr::NL / 2 : Gr::NL;
+    // runs of R consecutive scales (two runs per thread in the pair layouts)
+    constexpr int R = C::LAYOUT == kLayFull ? Gr::NL : Gr::NL / 2;
 #pragma unroll
     for (int r = 0; r < Gr::NL / R; ++r) {
       float* p = row + global_group<C, G>(t, r * R);
@@ -893,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     rotate_fwd<C, LAM>(xw, t, Y, lam);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
-    quantize<C, G>(Y, qw, sc);
+    quantize<C, G>(Y, qw, sc, t);
 
     const int o = int((ring.consumed - 1) % S_OUT);
     if (lane == 0) bulk_wait_read<S_OUT - 1>();
@@ -1086,7 +1131,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     rotate_fwd<C>(xw, t, Y);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
-    quantize<C, G>(Y, qw, sc);
+    quantize<C, G>(Y, qw, sc, t);
     store_codes<C>(qout, row, t, qw);
     const int64_t h = nt * C::VPW + row;
     if (h < a.n_heads) {
