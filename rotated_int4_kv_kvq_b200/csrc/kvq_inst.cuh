@@ -32,6 +32,15 @@ static __device__ unsigned g_status;
 #ifndef KVQ_SOUT_BIG
 #define KVQ_SOUT_BIG 1
 #endif
+#ifndef KVQ_SOUT_64
+#define KVQ_SOUT_64 2
+#endif
+// d = 64 SRFT 4-bit inverse with one scale per vector (g = 64): one output
+// tile in flight measured faster (88% against 85% of the copy peak, same
+// box); g = 32 measured slower (87% against 89%), SRHT the same.
+#ifndef KVQ_INV_SOUT_64_G64
+#define KVQ_INV_SOUT_64_G64 1
+#endif
 #ifndef KVQ_ATTN_MAX_CLUSTER
 #define KVQ_ATTN_MAX_CLUSTER 16
 #endif
@@ -59,8 +68,11 @@ struct Tuning {
   static constexpr int TPV = DefaultTPV<D>::value;
   static constexpr int FWD_STAGES = 2;
   static constexpr int INV_STAGES = D == 64 ? KVQ_INV_STAGES_64 : KVQ_INV_STAGES_BIG;
-  static constexpr int S_OUT = D == 64 ? 2 : KVQ_SOUT_BIG;
+  static constexpr int S_OUT = D == 64 ? KVQ_SOUT_64 : KVQ_SOUT_BIG;
   static constexpr bool SRFT = ROT == kRotSRFT;
+  template <int G, bool LAM, int BITS>
+  static constexpr int INV_S_OUT =
+      D == 64 && G == 64 && SRFT && !LAM && BITS == 4 ? KVQ_INV_SOUT_64_G64 : S_OUT;
   static constexpr int FWD_MINB =
       D == 64 ? (SRFT ? KVQ_FWD_MINB_64 : 4) : (D == 128 ? (SRFT ? KVQ_MINB_128_SRFT : 3)
                                         : (SRFT ? KVQ_FWD_MINB_256_SRFT : 3));
@@ -159,8 +171,11 @@ template <int D, int G, int ROT, bool LAM, int BITS = 4>
 cudaError_t inv_run(const InvLaunch& L) {
   using T = Tuning<D, ROT>;
   constexpr auto kern =
-      kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, T::INV_MINB, LAM, BITS>;
-  constexpr int smem = inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::S_OUT, BITS>();
+      kvq_inv_kernel<D, G, ROT, T::TPV, T::INV_STAGES, T::template INV_S_OUT<G, LAM, BITS>,
+                     T::INV_MINB, LAM, BITS>;
+  constexpr int smem =
+      inv_smem_bytes<D, G, ROT, T::TPV, T::INV_STAGES, T::template INV_S_OUT<G, LAM, BITS>,
+                     BITS>();
   int occ;
   unsigned* st;
   cudaError_t e = setup<kern>(smem, &occ);
