@@ -560,8 +560,8 @@ def run_suite(kvq, dev):
             out = torch.empty_like(x)
             algo = n * fwd_bytes(d, g)
             for rot in (kvq.SRFT, kvq.SRHT):
-                steps = 20
-                tot, f, i = time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 3)
+                steps = 50
+                tot, f, i = time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 5)
                 for name, ms in (("fwd", f), ("inv", i)):
                     us = 1e3 * ms / steps
                     res["sweep"].append({
