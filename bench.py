@@ -419,6 +419,10 @@ def main():
     }
     detail["fwd_frac"] = detail["fwd_algo_gbs"] / peak
     detail["inv_frac"] = detail["inv_algo_gbs"] / peak
+    # vectors per second: each direction alone, and through both per step
+    detail["fwd_vec_per_s"] = n / (fwd_ms * 1e-3 / args.steps)
+    detail["inv_vec_per_s"] = n / (inv_ms * 1e-3 / args.steps)
+    detail["vec_per_s"] = world * args.steps * n / (total_ms * 1e-3)
     # SRHT control on the same cache (context)
     t2, f2, i2 = time_kernels(kvq, x, packed, scales, out, signs, kvq.SRHT, g,
                               max(10, args.steps // 4), 3)
