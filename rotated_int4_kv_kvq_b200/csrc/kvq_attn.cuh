@@ -34,6 +34,7 @@ constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr int kAttnChunk = 32;   // tokens per staged chunk of a warp
 constexpr int kAttnStages = 2;   // chunks in flight per warp
+constexpr int kAttnMaxCluster = 16;  // blocks per KV head at most
 
 // Asynchronous global -> shared copies (cp.async); `bytes` < size zero-fills
 // the rest and 0 reads nothing.
@@ -359,25 +360,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
   if (threadIdx.x < 2 * NQ) s_part[threadIdx.x] = stage[threadIdx.x];
   cluster.sync();  // every block's triple is in its slot 0
 
-  // ---- block 0 merges the cluster and writes the output ----
-  if (rank == 0) {
-    // the merged accumulator goes to slot 1 of block 0
-    float* fin = s_part + AP::FLOATS;
-    for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
+  // ---- the cluster's blocks merge into slot 1 of block 0, a slice each ----
+  // weights of every block's triple per query: f_b / sum_b f_b l_b with
+  // f_b = 2^(m_b - max_b m_b); each block reads the (m, l) pairs once, one
+  // remote read per thread, and forms the weights in its own shared memory
+  __shared__ float s_w[kAttnMaxCluster * NQ];
+  __shared__ float s_l[kAttnMaxCluster * NQ];
+  for (int i = threadIdx.x; i < nblk * NQ; i += kAttnThreads) {
+    const float* src = cluster.map_shared_rank(s_part, i / NQ);
+    s_w[i] = src[2 * (i % NQ)];
+    s_l[i] = src[2 * (i % NQ) + 1];
+  }
+  __syncthreads();
+  if (threadIdx.x < NQ) {
+    const int qi = threadIdx.x;
+    float mm = -INFINITY;
+    for (int b = 0; b < nblk; ++b) mm = fmaxf(mm, s_w[b * NQ + qi]);
+    float ls = 0.0f;
+    for (int b = 0; b < nblk; ++b) {
+      const float mb = s_w[b * NQ + qi];
+      const float f = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
+      s_w[b * NQ + qi] = f;
+      ls += f * s_l[b * NQ + qi];
+    }
+    const float inv = 1.0f / ls;
+    for (int b = 0; b < nblk; ++b) s_w[b * NQ + qi] *= inv;
+  }
+  __syncthreads();
+  {
+    float* fin = cluster.map_shared_rank(s_part, 0) + AP::FLOATS;
+    constexpr int NE = NQ * D;
+    const int per = (NE + nblk - 1) / nblk;
+    const int e_end = (rank + 1) * per < NE ? (rank + 1) * per : NE;
+    for (int e = rank * per + threadIdx.x; e < e_end; e += kAttnThreads) {
       const int qi = e / D;
-      float mm = -INFINITY;
-      for (int b = 0; b < nblk; ++b) mm = fmaxf(mm, cluster.map_shared_rank(s_part, b)[2 * qi]);
-      float accv = 0.0f, ls = 0.0f;
-      for (int b = 0; b < nblk; ++b) {
-        const float* src = cluster.map_shared_rank(s_part, b);
-        const float f = src[2 * qi] == -INFINITY ? 0.0f : exp2f(src[2 * qi] - mm);
-        accv += f * src[2 * NQ + e];
-        ls += f * src[2 * qi + 1];
-      }
-      fin[2 * NQ + e] = accv / ls;
+      float accv = 0.0f;
+#pragma unroll 4
+      for (int b = 0; b < nblk; ++b)
+        accv += s_w[b * NQ + qi] * cluster.map_shared_rank(s_part, b)[2 * NQ + e];
+      fin[2 * NQ + e] = accv;
     }
   }
-  cluster.sync();  // remote reads done; other blocks may exit
+  cluster.sync();  // block 0's slot 1 is complete; remote reads done, others may exit
   if (rank == 0 && warp < a.nq) {
     const int qi = warp;
     const float* fin = s_part + AP::FLOATS + 2 * NQ + qi * D;

@@ -291,6 +291,7 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       // clusters of up to 16 blocks where the device can co-schedule them
+      static_assert(KVQ_ATTN_MAX_CLUSTER <= kAttnMaxCluster, "attention merge weights");
       int c = std::min(8, KVQ_ATTN_MAX_CLUSTER);
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
