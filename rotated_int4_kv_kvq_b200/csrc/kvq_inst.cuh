@@ -45,7 +45,7 @@ static __device__ unsigned g_status;
 #define KVQ_ATTN_MAX_CLUSTER 16
 #endif
 #ifndef KVQ_ATTN_ROWS_PER_WARP
-#define KVQ_ATTN_ROWS_PER_WARP 8
+#define KVQ_ATTN_ROWS_PER_WARP 4
 #endif
 #ifndef KVQ_FWD_MINB_64
 #define KVQ_FWD_MINB_64 5
