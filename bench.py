@@ -146,6 +146,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_min_mhz": min(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
@@ -447,7 +448,11 @@ def main():
 
     suite = None
     if args.suite and rank == 0:
+        suite_clock = ClockSampler(sampler.gpu)
+        suite_clock.start()
         suite = run_suite(kvq, dev)
+        suite_clock.stop()
+        suite["clocks"] = suite_clock.summary()  # over the whole suite
         with open(args.suite, "w") as f:
             json.dump(suite, f, indent=1)
 
@@ -564,8 +569,13 @@ def run_suite(kvq, dev):
             out = torch.empty_like(x)
             algo = n * fwd_bytes(d, g)
             for rot in (kvq.SRFT, kvq.SRHT):
-                steps = 50
-                tot, f, i = time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 5)
+                # median of three timed rounds (single rounds move by a few
+                # percent between boxes and runs)
+                steps = 20
+                rounds = [time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 3)
+                          for _ in range(3)]
+                f = statistics.median(r[1] for r in rounds)
+                i = statistics.median(r[2] for r in rounds)
                 for name, ms in (("fwd", f), ("inv", i)):
                     us = 1e3 * ms / steps
                     res["sweep"].append({
