@@ -39,7 +39,11 @@
  *     per-call state.
  *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
  *     return as soon as the work is enqueued.  Results are ready when the
- *     stream is synchronized.
+ *     stream is synchronized.  The decode-step and attention calls are
+ *     launched with programmatic dependent launch: their blocks may be
+ *     scheduled while the previous kernel of the stream drains, but they
+ *     touch no global memory before that kernel has completed, so stream
+ *     order holds for their inputs and outputs as for any other launch.
  *   - Every argument check runs on the host before anything is launched; a
  *     failing check returns its status and enqueues nothing.  KVQ_ERR_CUDA
  *     reports a CUDA runtime error raised while enqueueing.

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
   using AP = AttnPartial<D, NQ>;
   extern __shared__ __align__(16) float s_part[];  // staging rings, then merge slots
 
+  pdl_wait();  // no global access before the previous kernel completes
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
   const int nblk = int(cluster.num_blocks());
@@ -319,6 +320,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
     issue(c + kAttnStages);
   }
   cp_async_wait<0>();
+  pdl_release();
   __syncthreads();  // the staging rings become the merge area
 
   // ---- merge the warps of this block ----

@@ -1094,6 +1094,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t bars = smem_u32(&bars_sm[warp][0]);
   const uint32_t bar_new = bars + 8u * S_IN;
 
+  pdl_wait();  // no global access before the previous kernel completes
   fill_sign_masks<C>(a.signs, s_mask);
   if (lane == 0) {
     for (int s = 0; s <= S_IN; ++s) mbar_init(bars + 8u * s, 1);
@@ -1227,6 +1228,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
       bulk_commit();
     }
   }
+  pdl_release();
   if (lane == 0) {
     bulk_wait_all();
     if (failed) drain_and_fail<S_IN>(bars, ring, status);

@@ -16,6 +16,11 @@
 
 #include <type_traits>
 
+// Decode-path kernels use programmatic dependent launch (0 disables it).
+#ifndef KVQ_PDL
+#define KVQ_PDL 1
+#endif
+
 namespace kvq {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -223,6 +228,29 @@ __device__ __forceinline__ void bulk_wait_read() {
 
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialization may start while the kernel before it in the stream is
+// still finishing; pdl_wait() returns once that kernel has completed and its
+// memory operations are visible (at once for a launch without the
+// attribute), so every global access of such a kernel comes after it.
+// pdl_release() lets the next kernel of the stream begin launching its
+// blocks once every block of this one has released or exited; it does not
+// make any of this kernel's results visible to it.  The decode-path kernels
+// release after their main loop: released at kernel entry, the next
+// kernel's blocks were placed while this one's were still running and the
+// 26-call decode step measured slower at some lengths (1025 rows: 88 us
+// against 76 us released late, 86 us without the attribute).
+__device__ __forceinline__ void pdl_wait() {
+#if KVQ_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+__device__ __forceinline__ void pdl_release() {
+#if KVQ_PDL
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {

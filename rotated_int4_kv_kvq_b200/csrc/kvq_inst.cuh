@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "kvq_codec.cuh"
 #include "kvq_attn.cuh"
@@ -131,6 +132,31 @@ cudaError_t setup(int smem, int* occ_out) {
   return cudaSuccess;
 }
 
+// Launch attribute of the decode-path kernels: programmatic stream
+// serialization, so that a kernel's blocks can be scheduled while the
+// previous kernel of the stream drains (the kernels wait for it with
+// griddepcontrol.wait before touching global memory).
+inline void pdl_attribute(cudaLaunchAttribute& at) {
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = KVQ_PDL ? 1 : 0;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, int smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid), 1, 1);
+  cfg.blockDim = dim3(unsigned(threads), 1, 1);
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  pdl_attribute(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 inline int grid_for(int64_t n_tiles, int sm_count, int occ) {
   const int64_t want = (n_tiles + kWarps - 1) / kWarps;
   return int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count) * occ)));
@@ -221,9 +247,8 @@ cudaError_t decode_one(const DecodeLaunch& L) {
   a.n_new_tiles = (L.n_heads + vpw - 1) / vpw;
   a.tok_tiles = (L.pos + vpw - 1) / vpw;
   a.n_tiles = a.n_new_tiles + L.n_heads * a.tok_tiles;
-  kern<<<grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream>>>(
-      *L.tmXn, *L.tmQn, *L.tmOn, *L.tmQc, *L.tmOc, a, st);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid_for(a.n_tiles, L.sm_count, occ), kThreads, smem, L.stream,
+                    *L.tmXn, *L.tmQn, *L.tmOn, *L.tmQc, *L.tmOc, a, st);
 }
 
 // Resident 256-thread blocks per SM of a one-warp-per-vector kernel (cached
@@ -258,8 +283,8 @@ cudaError_t decode_wide_one(const DecodeWideLaunch& L) {
   cudaError_t e = wide_occupancy<kern>(&occ);
   if (e != cudaSuccess) return e;
   DecodeWideArgs a{L.x_new, L.packed, L.scales, L.out, L.signs, L.n_heads, L.cap, L.pos};
-  kern<<<wide_grid(L.n_heads * (L.pos + 1), L.sm_count, occ), kWideThreads, 0, L.stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, wide_grid(L.n_heads * (L.pos + 1), L.sm_count, occ), kWideThreads, 0,
+                    L.stream, a);
 }
 
 template <int D, int G, int ROT>
@@ -271,8 +296,7 @@ cudaError_t window_one(const WindowLaunch& L) {
   WindowArgs a{L.x_new, L.packed, L.scales, L.kv, L.signs, L.n_heads, L.cap, L.pos, L.window};
   const bool flush = (L.pos + 1) % L.window == 0;
   const int64_t rows = flush ? L.n_heads * L.window : L.n_heads;
-  kern<<<wide_grid(rows, L.sm_count, occ), kWideThreads, 0, L.stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, wide_grid(rows, L.sm_count, occ), kWideThreads, 0, L.stream, a);
 }
 
 template <int D, int ROT, int NQ>
@@ -322,13 +346,14 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   cfg.blockDim = dim3(kAttnThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = L.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(cl);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  pdl_attribute(attr[0]);
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = unsigned(cl);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cl > 1 ? 1 : 0;  // a one-block cluster needs no cluster launch
+  cfg.numAttrs = cl > 1 ? 2 : 1;  // a one-block cluster needs no cluster launch
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
   return e == cudaSuccess ? cudaGetLastError() : e;
 }

@@ -439,6 +439,7 @@ __global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const Dec
   constexpr int NG = D / G;
   constexpr int GL = G / Wide<D, ROT>::W;  // lanes (chunks) per group
   const int lane = threadIdx.x & 31;
+  pdl_wait();  // no global access before the previous kernel completes
   WideLane<D, ROT> L;
   L.init(a.signs, lane);
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -477,6 +478,7 @@ __global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const Dec
     }
     wide_dequant_row<D, ROT>(code, s, a.out + (head * (a.pos + 1) + row) * D, L);
   }
+  pdl_release();
 }
 
 // ------------------------------------------- windowed decode (prefix cache) ---
@@ -504,12 +506,14 @@ __global__ void __launch_bounds__(kWideThreads) kvq_window_wide_kernel(const Win
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const bool flush = (a.pos + 1) % a.window == 0;
+  pdl_wait();  // no global access before the previous kernel completes
   if (!flush) {  // copy the new rows into the tail
     for (int64_t h = gw; h < a.n_heads; h += nw) {
       const uint4* src = reinterpret_cast<const uint4*>(a.x_new + h * D);
       uint4* dst = reinterpret_cast<uint4*>(a.kv + (h * a.cap + a.pos) * D);
       for (int c = lane; c < D / 8; c += 32) dst[c] = __ldg(src + c);
     }
+    pdl_release();
     return;
   }
   WideLane<D, ROT> L;
@@ -528,6 +532,7 @@ __global__ void __launch_bounds__(kWideThreads) kvq_window_wide_kernel(const Win
     __syncwarp();  // every lane has read the source row before it is overwritten
     wide_dequant_row<D, ROT>(code, s, a.kv + (head * a.cap + row) * D, L);
   }
+  pdl_release();
 }
 
 }  // namespace kvq
