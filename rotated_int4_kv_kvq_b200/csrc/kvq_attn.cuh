@@ -339,24 +339,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
       dst[1] = hi2(acc[qi][j]);
     }
   __syncthreads();
-  // thread i of the block merges element i of every (query, coordinate) and
-  // leaves the block's triple in warp slot 0
-  for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
-    const int qi = e / D;
+  // per query, the weight f_w = 2^(m_w - max_w m_w) of every warp's partial,
+  // formed once; then thread i merges element i of every (query,
+  // coordinate) and leaves the block's triple in warp slot 0
+  __shared__ float s_bw[kAttnWarps * NQ];
+  if (threadIdx.x < NQ) {
+    const int qi = threadIdx.x;
     float mm = -INFINITY;
     for (int w = 0; w < kAttnWarps; ++w) mm = fmaxf(mm, s_part[w * AP::FLOATS + 2 * qi]);
-    float accv = 0.0f, ls = 0.0f;
+    float ls = 0.0f;
     for (int w = 0; w < kAttnWarps; ++w) {
       const float* src = s_part + w * AP::FLOATS;
       const float f = src[2 * qi] == -INFINITY ? 0.0f : exp2f(src[2 * qi] - mm);
-      accv += f * src[2 * NQ + e];
+      s_bw[w * NQ + qi] = f;
       ls += f * src[2 * qi + 1];
     }
+    stage[2 * qi] = mm;  // m, l of every slot are still being read: stage them
+    stage[2 * qi + 1] = ls;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
+    const int qi = e / D;
+    float accv = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w)
+      accv += s_bw[w * NQ + qi] * s_part[w * AP::FLOATS + 2 * NQ + e];
     s_part[2 * NQ + e] = accv;  // slot 0 (warp 0's region): read only by this thread
-    if (e % D == 0) {  // m, l of every slot are still being read: stage them
-      stage[2 * qi] = mm;
-      stage[2 * qi + 1] = ls;
-    }
   }
   __syncthreads();
   if (threadIdx.x < 2 * NQ) s_part[threadIdx.x] = stage[threadIdx.x];
