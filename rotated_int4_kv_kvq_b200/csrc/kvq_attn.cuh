@@ -340,22 +340,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
     }
   __syncthreads();
   // per query, the weight f_w = 2^(m_w - max_w m_w) of every warp's partial,
-  // formed once; then thread i merges element i of every (query,
+  // formed once (warp qi for query qi, lane w for warp w's partial, max and
+  // sum by shuffles); then thread i merges element i of every (query,
   // coordinate) and leaves the block's triple in warp slot 0
   __shared__ float s_bw[kAttnWarps * NQ];
-  if (threadIdx.x < NQ) {
-    const int qi = threadIdx.x;
-    float mm = -INFINITY;
-    for (int w = 0; w < kAttnWarps; ++w) mm = fmaxf(mm, s_part[w * AP::FLOATS + 2 * qi]);
-    float ls = 0.0f;
-    for (int w = 0; w < kAttnWarps; ++w) {
-      const float* src = s_part + w * AP::FLOATS;
-      const float f = src[2 * qi] == -INFINITY ? 0.0f : exp2f(src[2 * qi] - mm);
-      s_bw[w * NQ + qi] = f;
-      ls += f * src[2 * qi + 1];
+  static_assert(NQ <= kAttnWarps && kAttnWarps <= 32, "one warp per query, a lane per warp");
+  if (warp < NQ) {
+    const int qi = warp;
+    const bool has = lane < kAttnWarps;
+    const float mw = has ? s_part[lane * AP::FLOATS + 2 * qi] : -INFINITY;
+    const float lw = has ? s_part[lane * AP::FLOATS + 2 * qi + 1] : 0.0f;
+    float mm = mw;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
+    const float f = mw == -INFINITY ? 0.0f : exp2f(mw - mm);
+    float ls = f * lw;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+    if (has) s_bw[lane * NQ + qi] = f;
+    if (lane == 0) {  // m, l of every slot are still being read: stage them
+      stage[2 * qi] = mm;
+      stage[2 * qi + 1] = ls;
     }
-    stage[2 * qi] = mm;  // m, l of every slot are still being read: stage them
-    stage[2 * qi + 1] = ls;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
@@ -382,19 +388,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
     s_l[i] = src[2 * (i % NQ) + 1];
   }
   __syncthreads();
-  if (threadIdx.x < NQ) {
-    const int qi = threadIdx.x;
-    float mm = -INFINITY;
-    for (int b = 0; b < nblk; ++b) mm = fmaxf(mm, s_w[b * NQ + qi]);
-    float ls = 0.0f;
-    for (int b = 0; b < nblk; ++b) {
-      const float mb = s_w[b * NQ + qi];
-      const float f = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
-      s_w[b * NQ + qi] = f;
-      ls += f * s_l[b * NQ + qi];
-    }
-    const float inv = 1.0f / ls;
-    for (int b = 0; b < nblk; ++b) s_w[b * NQ + qi] *= inv;
+  static_assert(kAttnMaxCluster <= 32, "a lane per block of the cluster");
+  if (warp < NQ) {  // warp qi: lane b forms block b's weight, max and sum by shuffles
+    const int qi = warp;
+    const bool has = lane < nblk;
+    const float mb = has ? s_w[lane * NQ + qi] : -INFINITY;
+    const float lb = has ? s_l[lane * NQ + qi] : 0.0f;
+    float mm = mb;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
+    const float f = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
+    float ls = f * lb;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+    if (has) s_w[lane * NQ + qi] = f * (1.0f / ls);
   }
   __syncthreads();
   {
