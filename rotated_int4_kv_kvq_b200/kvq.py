@@ -9,6 +9,7 @@ module fails if libkvq.so has not been built
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -86,10 +87,37 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> int | None:
+def _stream(stream, dev: torch.device) -> int | None:
+    """Raw handle of `stream`; None means the current stream of `dev`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
     return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _device_of(tensors, stream) -> torch.device:
+    """The one CUDA device that every tensor argument lives on.
+
+    The library launches on the calling thread's current device and builds
+    its copy descriptors over the pointers it is given, so all operands of a
+    call must share one device; an explicit torch stream must belong to it
+    too.  Raises ValueError before anything is launched otherwise.  (A raw
+    integer stream handle cannot be checked here; it must belong to the same
+    device.)"""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError("all tensor arguments must be on one CUDA device, got "
+                         + ", ".join(sorted(str(d) for d in devs)))
+    dev = devs.pop()
+    if isinstance(stream, torch.cuda.Stream) and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, tensors on {dev}")
+    return dev
+
+
+def _current(dev: torch.device):
+    """Context that makes `dev` the current device for one library call."""
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
 
 
 def _check(t: torch.Tensor, name: str, dtype, shape):
@@ -125,15 +153,18 @@ def kvq_rot_quant_fwd(x: torch.Tensor, signs: torch.Tensor, rot: int, group: int
         scales = torch.empty((n, d // group), dtype=torch.float32, device=x.device)
     _check(packed, "packed", torch.uint8, (n, d // 2))
     _check(scales, "scales", torch.float32, (n, d // group))
-    if lam is None:
-        st = lib.kvq_rot_quant_fwd(_ptr(x), n, d, group, _ptr(signs), rot, _ptr(packed),
-                                   _ptr(scales), _stream(stream))
-        _raise("kvq_rot_quant_fwd", st)
-    else:
+    if lam is not None:
         _check(lam, "lam", torch.float32, (d,))
-        st = lib.kvq_rot_quant_fwd_lambda(_ptr(x), n, d, group, _ptr(signs), _ptr(lam), rot,
-                                          _ptr(packed), _ptr(scales), _stream(stream))
-        _raise("kvq_rot_quant_fwd_lambda", st)
+    dev = _device_of((x, signs, packed, scales, lam), stream)
+    with _current(dev):
+        if lam is None:
+            st = lib.kvq_rot_quant_fwd(_ptr(x), n, d, group, _ptr(signs), rot, _ptr(packed),
+                                       _ptr(scales), _stream(stream, dev))
+            _raise("kvq_rot_quant_fwd", st)
+        else:
+            st = lib.kvq_rot_quant_fwd_lambda(_ptr(x), n, d, group, _ptr(signs), _ptr(lam), rot,
+                                              _ptr(packed), _ptr(scales), _stream(stream, dev))
+            _raise("kvq_rot_quant_fwd_lambda", st)
     return packed, scales
 
 
@@ -151,16 +182,19 @@ def kvq_dequant_rot_inv(packed: torch.Tensor, scales: torch.Tensor, signs: torch
     if out is None:
         out = torch.empty((n, d), dtype=torch.float16, device=packed.device)
     _check(out, "out", torch.float16, (n, d))
-    if lam is None:
-        st = lib.kvq_dequant_rot_inv(_ptr(packed), _ptr(scales), n, d, group, _ptr(signs), rot,
-                                     _ptr(out), _stream(stream))
-        _raise("kvq_dequant_rot_inv", st)
-    else:
+    if lam is not None:
         _check(lam, "lam", torch.float32, (d,))
-        st = lib.kvq_dequant_rot_inv_lambda(_ptr(packed), _ptr(scales), n, d, group,
-                                            _ptr(signs), _ptr(lam), rot, _ptr(out),
-                                            _stream(stream))
-        _raise("kvq_dequant_rot_inv_lambda", st)
+    dev = _device_of((packed, scales, signs, out, lam), stream)
+    with _current(dev):
+        if lam is None:
+            st = lib.kvq_dequant_rot_inv(_ptr(packed), _ptr(scales), n, d, group, _ptr(signs),
+                                         rot, _ptr(out), _stream(stream, dev))
+            _raise("kvq_dequant_rot_inv", st)
+        else:
+            st = lib.kvq_dequant_rot_inv_lambda(_ptr(packed), _ptr(scales), n, d, group,
+                                                _ptr(signs), _ptr(lam), rot, _ptr(out),
+                                                _stream(stream, dev))
+            _raise("kvq_dequant_rot_inv_lambda", st)
     return out
 
 
@@ -179,8 +213,10 @@ def kvq_rot_quant_fwd_bits(x: torch.Tensor, signs: torch.Tensor, rot: int, group
         scales = torch.empty((n, d // group), dtype=torch.float32, device=x.device)
     _check(packed, "packed", torch.uint8, (n, qp))
     _check(scales, "scales", torch.float32, (n, d // group))
-    st = lib.kvq_rot_quant_fwd_bits(_ptr(x), n, d, group, bits, _ptr(signs), rot, _ptr(packed),
-                                    _ptr(scales), _stream(stream))
+    dev = _device_of((x, signs, packed, scales), stream)
+    with _current(dev):
+        st = lib.kvq_rot_quant_fwd_bits(_ptr(x), n, d, group, bits, _ptr(signs), rot,
+                                        _ptr(packed), _ptr(scales), _stream(stream, dev))
     _raise("kvq_rot_quant_fwd_bits", st)
     return packed, scales
 
@@ -197,8 +233,10 @@ def kvq_dequant_rot_inv_bits(packed: torch.Tensor, scales: torch.Tensor, signs: 
     if out is None:
         out = torch.empty((n, d), dtype=torch.float16, device=packed.device)
     _check(out, "out", torch.float16, (n, d))
-    st = lib.kvq_dequant_rot_inv_bits(_ptr(packed), _ptr(scales), n, d, group, bits, _ptr(signs),
-                                      rot, _ptr(out), _stream(stream))
+    dev = _device_of((packed, scales, signs, out), stream)
+    with _current(dev):
+        st = lib.kvq_dequant_rot_inv_bits(_ptr(packed), _ptr(scales), n, d, group, bits,
+                                          _ptr(signs), rot, _ptr(out), _stream(stream, dev))
     _raise("kvq_dequant_rot_inv_bits", st)
     return out
 
@@ -217,8 +255,10 @@ def kvq_decode_step(x_new: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
     if out is None:
         out = torch.empty((h, pos + 1, d), dtype=torch.float16, device=x_new.device)
     _check(out, "out", torch.float16, (h, pos + 1, d))
-    st = lib.kvq_decode_step(_ptr(x_new), _ptr(packed), _ptr(scales), h, cap, pos, d, group,
-                             _ptr(signs), rot, _ptr(out), _stream(stream))
+    dev = _device_of((x_new, packed, scales, signs, out), stream)
+    with _current(dev):
+        st = lib.kvq_decode_step(_ptr(x_new), _ptr(packed), _ptr(scales), h, cap, pos, d, group,
+                                 _ptr(signs), rot, _ptr(out), _stream(stream, dev))
     _raise("kvq_decode_step", st)
     return out
 
@@ -237,8 +277,11 @@ def kvq_decode_step_windowed(x_new: torch.Tensor, packed: torch.Tensor, scales: 
     _check(scales, "scales", torch.float32, (h, cap, d // group))
     _check(kv, "kv", torch.float16, (h, cap, d))
     _check(signs, "signs", torch.int8, (d,))
-    st = lib.kvq_decode_step_windowed(_ptr(x_new), _ptr(packed), _ptr(scales), _ptr(kv), h, cap,
-                                      pos, window, d, group, _ptr(signs), rot, _stream(stream))
+    dev = _device_of((x_new, packed, scales, kv, signs), stream)
+    with _current(dev):
+        st = lib.kvq_decode_step_windowed(_ptr(x_new), _ptr(packed), _ptr(scales), _ptr(kv), h,
+                                          cap, pos, window, d, group, _ptr(signs), rot,
+                                          _stream(stream, dev))
     _raise("kvq_decode_step_windowed", st)
     return kv
 
@@ -262,9 +305,11 @@ def kvq_attend_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.T
         out = torch.empty((h, nq, d), dtype=torch.float16, device=q.device)
     _check(out, "out", torch.float16, (h, nq, d))
     scale = float(sm_scale) if sm_scale is not None else d ** -0.5
-    st = lib.kvq_attend_decode(_ptr(q), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
-                               _ptr(v_scales), h, nq, cap, length, d, group, _ptr(signs), rot,
-                               scale, _ptr(out), _stream(stream))
+    dev = _device_of((q, k_packed, k_scales, v_packed, v_scales, signs, out), stream)
+    with _current(dev):
+        st = lib.kvq_attend_decode(_ptr(q), _ptr(k_packed), _ptr(k_scales), _ptr(v_packed),
+                                   _ptr(v_scales), h, nq, cap, length, d, group, _ptr(signs),
+                                   rot, scale, _ptr(out), _stream(stream, dev))
     _raise("kvq_attend_decode", st)
     return out
 

@@ -161,3 +161,45 @@ def test_bits_host_checks(kvq):
     assert fwd(A, 10, 96, 32, 8, A, 0, A, A, None) == 2
     assert fwd(A, 0, 128, 32, 3, A, 0, A, A, None) == 0
     assert inv(A, A, 0, 64, 64, 6, A, 1, A, None) == 0
+
+
+def test_operands_on_different_devices_are_rejected_before_launch(kvq):
+    import torch
+    a = torch.empty(4, device="cpu")
+    b = torch.empty(4, device="meta")
+    with pytest.raises(ValueError, match="one CUDA device"):
+        kvq._device_of((a, b, None), None)
+    assert kvq._device_of((a, None, a), None) == a.device
+
+
+def test_non_cuda_tensors_are_rejected_before_launch(kvq):
+    import torch
+    x = torch.zeros((32, 64), dtype=torch.float16)
+    signs = torch.ones(64, dtype=torch.int8)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        kvq.kvq_rot_quant_fwd(x, signs, kvq.SRFT, 64)
+
+
+@pytest.mark.gpu
+def test_calls_run_on_the_tensors_device(kvq):
+    """Operands on one device other than the current one run there; operands
+    split over two devices, or a stream of another device, raise before any
+    launch."""
+    import torch
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two CUDA devices")
+    d, g = 64, 64
+    x1 = torch.randn((64, d), device="cuda:1").half()
+    s1 = torch.ones(d, dtype=torch.int8, device="cuda:1")
+    with torch.cuda.device(0):
+        p1, sc1 = kvq.kvq_rot_quant_fwd(x1, s1, kvq.SRFT, g)
+        torch.cuda.synchronize(1)
+    with torch.cuda.device(1):
+        p_ref, sc_ref = kvq.kvq_rot_quant_fwd(x1, s1, kvq.SRFT, g)
+        torch.cuda.synchronize(1)
+    assert torch.equal(p1, p_ref) and torch.equal(sc1, sc_ref)
+    s0 = s1.to("cuda:0")
+    with pytest.raises(ValueError, match="one CUDA device"):
+        kvq.kvq_rot_quant_fwd(x1, s0, kvq.SRFT, g)
+    with pytest.raises(ValueError, match="stream"):
+        kvq.kvq_rot_quant_fwd(x1, s1, kvq.SRFT, g, stream=torch.cuda.Stream(device=0))
