@@ -3,22 +3,28 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
                     [--suite PATH]
 
-One step = the whole hot path over one synthetic SmolLM2-1.7B-shaped KV cache
-(24 layers x K,V x 32 kv heads x 4096 tokens x d=64, group 64, SRFT): the
-forward kernel (x -> packed codes + scales) then the inverse kernel
-(codes + scales -> x_hat).  The cache (805 MB of fp16) is larger than L2, so
-no flush is needed between steps.  Metric: GB/s of fp16 KV through the two
-kernels (2 * n_vec * d * 2 bytes per step), device-timed with CUDA events.
+Workload: the large-batch throughput sweep.  K and V of 64 sequences x 8 kv
+heads x 8192 tokens (8,388,608 vectors) for every d in {64, 128, 256}, fp16
+N(0, 1) with 4 outlier channels per head x20, groups g in {32, d}.  One step
+runs every cell of the sweep once: for each d, each g and each rotation
+(SRFT, then the SRHT control) the forward kernel (x -> packed codes + scales)
+then the inverse kernel (codes + scales -> x_hat), 24 launches over 7.5 GB of
+fp16 inputs, all resident in HBM and larger than L2 (no flush is needed
+between launches).  Metric: GB/s of fp16 KV through the kernels (n_vec * d * 2
+bytes per launch), device-timed with CUDA events; every cell is also reported
+with its best and median launch time and its algorithmic HBM bytes
+(2d + d/2 + 4d/g per vector) as a fraction of the measured copy peak.
 
-Under torchrun each rank runs the same workload on its own GPU (independent
-shards, no collective on the data path: weak scaling); rank 0 prints one JSON
-line with the whole-job value (sum over ranks / max time over ranks).
+Under torchrun (or `--gpus N`, which starts torchrun itself) each rank runs
+the same sweep on its own GPU (independent shards, no collective on the data
+path: weak scaling); rank 0 prints one JSON line with the whole-job value
+(bytes of all ranks / max time over ranks).
 
 --impl reference times the CPU oracle (the plain float64 restatement of the
-method) on a bounded sample of the same workload on the host cores.
---suite PATH additionally measures every (d, group, rotation, direction) of
-the large-batch sweep and the Gemma-3-1B decode-step latency, and writes them
-as JSON to PATH.
+method) on a bounded sample of the same sweep on the host cores.
+--suite PATH additionally measures the other code widths, the lambda hook,
+the eager decode step and the int4-reading attention, and writes them as
+JSON to PATH.
 """
 
 from __future__ import annotations
@@ -27,6 +33,7 @@ import argparse
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -45,6 +52,13 @@ METRIC = "fp16 KV GB/s through fused rotate+int4 quant / dequant+inverse; % of H
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "rotated_int4_kv_kvq_b200", "csrc")
+
+SWEEP_D = (64, 128, 256)
+ROTS = ((0, "srft"), (1, "srht"))
+
+
+def sweep_groups(d):
+    return (32, d)
 
 
 # the sources the tiled forward / inverse kernels are built and launched from
@@ -72,9 +86,15 @@ def fwd_bytes(d, g):  # algorithmic bytes per vector, forward (inverse: same)
     return 2 * d + d // 2 + 4 * (d // g)
 
 
+def cell_name(d, g, rot, direction):
+    kern = "kvq_fwd_kernel" if direction == "fwd" else "kvq_inv_kernel"
+    return f"{kern} d={d} g={g} {ROTS[rot][1]}"
+
+
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
-    was taken on the current kernel sources (else None)."""
+    """DRAM bytes per full-size launch of `kernel` (a cell name) from the
+    committed ncu summary, if it was taken on the current kernel sources
+    (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -87,8 +107,27 @@ def recorded_traffic(kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+# --------------------------------------------------------------- clocks ---
+
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def summarize_clocks(samples, source):
+    """samples: (sm_mhz, max_mhz, set of active reason names) per sample."""
+    sm = [s[0] for s in samples]
+    mx = [s[1] for s in samples]
+    reasons = set()
+    for s in samples:
+        reasons |= s[2]
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_min_mhz": min(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+            "samples": len(sm), "source": source}
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms (the
+    fallback when NVML cannot be read from Python)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -126,29 +165,121 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.lines:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, 1e30)
         rows = [l for (t, l) in self.lines if t0 - 0.25 <= t <= t1 + 0.25] or \
             [l for (_, l) in self.lines]
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        samples = []
         for r in rows:
             f = [c.strip() for c in r.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                sm, mx = float(f[1]), float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_min_mhz": min(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            act = {n for n, v in zip(REASON_NAMES, f[5:9]) if v.lower().startswith("active")}
+            samples.append((sm, mx, act))
+        return summarize_clocks(samples, "nvidia-smi 200 ms")
+
+
+class NvmlSampler:
+    """Read-only NVML polling of the SM clock and the clock-event reasons
+    every `period` seconds from a background thread (changes no setting).
+    Only samples between the first two mark() calls are summarized."""
+
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+            "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, handle, nvml, period=0.01):
+        self.h, self.nvml, self.period = handle, nvml, period
+        self.samples = []
+        self.marks = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+        self.max_mhz = float(nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM))
+
+    def _reasons(self):
+        fn = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _loop(self):
+        while not self.stop_flag.is_set():
+            try:
+                sm = float(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                bits = int(self._reasons())
+                act = {n for n, b in self.BITS.items() if bits & b}
+                self.samples.append((time.time(), sm, act))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        t0, t1 = (self.marks[0], self.marks[1]) if len(self.marks) >= 2 else (0, 1e30)
+        rows = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+        return summarize_clocks([(sm, self.max_mhz, act) for (_, sm, act) in rows],
+                                f"nvml {int(self.period * 1000)} ms")
+
+
+def make_sampler(dev: torch.device):
+    """NVML sampler for the CUDA device `dev` (matched by UUID), else the
+    nvidia-smi sampler."""
+    try:
+        import pynvml as nvml
+        nvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        h = nvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        return NvmlSampler(h, nvml)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        idx = dev.index or 0
+        gpu = int(vis[idx]) if idx < len(vis) and vis[idx].isdigit() else idx
+        return ClockSampler(gpu)
+
+
+# ------------------------------------------------------------- launching ---
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_command(argv, gpus, port):
+    """torchrun command line that runs this script on `gpus` ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            "--nproc-per-node", str(gpus), "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def maybe_relaunch(args, argv):
+    """--gpus N > 1 outside torchrun: start N ranks under torchrun and exit
+    with its status.  Inside torchrun, --gpus must equal WORLD_SIZE."""
+    world = os.environ.get("WORLD_SIZE")
+    if world is not None:
+        if int(world) != args.gpus:
+            sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
+        return
+    if args.gpus <= 1:
+        return
+    if args.impl == "kvq":
+        visible = torch.cuda.device_count() if torch.cuda.is_available() else 0
+        if visible < args.gpus:
+            sys.exit(f"bench.py: --gpus {args.gpus} but {visible} CUDA device(s) are visible")
+    r = subprocess.run(relaunch_command(argv, args.gpus, _free_port()))
+    sys.exit(r.returncode)
 
 
 def dist_setup():
@@ -190,133 +321,147 @@ def cpu_threads() -> int:
         return 1
 
 
-def oracle_sample_gbs(x_sample: np.ndarray, signs, rot, group, min_seconds: float,
-                      chunk: int = 1 << 16):
-    """Oracle fwd + inv over chunks of the sample until `min_seconds` pass.
-    Returns (GB/s of fp16 KV, vectors processed, seconds)."""
-    import oracle.kvq_oracle as O
-    d = x_sample.shape[1]
-    done, t0 = 0, time.perf_counter()
-    i = 0
-    while True:
-        part = x_sample[(i * chunk) % len(x_sample):][:chunk]
-        p, s = O.rot_quant_fwd(part, signs, rot, group)
-        O.dequant_rot_inv(p, s, signs, rot, group)
-        done += len(part)
-        i += 1
-        el = time.perf_counter() - t0
-        if el >= min_seconds:
-            break
-    return 2 * done * d * 2 / el / 1e9, done, el
+# ------------------------------------------------------------- workload ---
+
+def workload_desc():
+    return ("large-batch sweep: K,V x 64 seq x 8 kv heads x 8192 tokens (8,388,608 vectors) "
+            "for d in {64,128,256}, fp16 N(0,1) + 4 outlier channels/head x20, g in {32, d}, "
+            "SRFT and SRHT, forward then inverse: 24 launches per step")
 
 
-def headline_shape():
-    return W.config(2)
+class SweepData:
+    """Device tensors of one d of the sweep: x, out, packed and one scales
+    tensor per group."""
+
+    def __init__(self, d, dev, seed_offset=0):
+        shape = W.config(5, d=d, group=32)
+        self.d = d
+        self.x = W.make_kv(shape, device=dev, seed=shape.seed + seed_offset)
+        self.n = self.x.shape[0]
+        self.signs = torch.from_numpy(W.make_signs(d)).to(dev)
+        self.packed = torch.empty((self.n, d // 2), dtype=torch.uint8, device=dev)
+        self.scales = {g: torch.empty((self.n, d // g), dtype=torch.float32, device=dev)
+                       for g in sweep_groups(d)}
+        self.out = torch.empty_like(self.x)
 
 
-def workload_desc(shape):
-    return (f"{shape.name}: {shape.layers} layers x K,V x {shape.heads} kv heads x "
-            f"{shape.tokens} tokens x d={shape.d} fp16, group {shape.group}, SRFT, "
-            f"forward then inverse over the whole cache")
+def sweep_cells():
+    """(d, g, rot) in execution order; each runs forward then inverse."""
+    return [(d, g, rot) for d in SWEEP_D for g in sweep_groups(d) for rot, _ in ROTS]
 
 
-def run_reference(args, world, rank):
-    if rank != 0:
-        return
-    import oracle.kvq_oracle as O
-    shape = headline_shape()
-    d, g = shape.d, shape.group
-    small = W.scaled(shape, layers=1, heads=4)  # 32768 vectors of the same recipe
-    x = W.make_kv(small).numpy()
-    signs = W.make_signs(d)
-    per_step = 1 << 14
-    times = []
-    for k in range(args.warmup + args.steps):
-        part = x[(k * per_step) % len(x):][:per_step]
-        t0 = time.perf_counter()
-        p, s = O.rot_quant_fwd(part, signs, O.SRFT, g)
-        O.dequant_rot_inv(p, s, signs, O.SRFT, g)
-        dt = time.perf_counter() - t0
-        if k >= args.warmup:
-            times.append(dt)
-    total = sum(times)
-    value = 2 * per_step * d * 2 * len(times) / total / 1e9
-    cores = cpu_threads()
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(shape) + f" (CPU oracle: {per_step} vectors per step)",
-                   "n_vec_per_step": per_step, "d": d, "group": g, "rot": "srft"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{per_step} vectors per step of the {shape.name} recipe"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
+def sweep_fp16_bytes_per_step(n_by_d):
+    """fp16 KV bytes one step moves through the kernels (both directions)."""
+    return sum(2 * n_by_d[d] * d * 2 for (d, g, rot) in sweep_cells())
 
 
-def time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, warmup, sampler=None,
-                 lam=None):
-    """Device time of `steps` fwd+inv passes; per-kernel sums via events.
-    With `lam`, the per-channel lambda entry points."""
+def time_sweep(kvq, S, steps, warmup, sampler=None):
+    """Device time of `steps` sweep steps; per-launch times of every cell.
+    Returns (total_ms, {(d, g, rot, dir): [ms per launch]})."""
     stream = torch.cuda.current_stream()
+    cells = sweep_cells()
+
+    def launch(d, g, rot, direction):
+        T = S[d]
+        if direction == "fwd":
+            kvq.kvq_rot_quant_fwd(T.x, T.signs, rot, g, T.packed, T.scales[g], stream)
+        else:
+            kvq.kvq_dequant_rot_inv(T.packed, T.scales[g], T.signs, rot, g, T.out, stream)
+
     for _ in range(warmup):
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream, lam=lam)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream, lam=lam)
+        for (d, g, rot) in cells:
+            launch(d, g, rot, "fwd")
+            launch(d, g, rot, "inv")
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    n_launch = 2 * len(cells)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
+          for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if sampler:
         sampler.mark()
     start.record(stream)
     for k in range(steps):
+        i = 0
         ev[k][0].record(stream)
-        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream, lam=lam)
-        ev[k][1].record(stream)
-        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream, lam=lam)
-        ev[k][2].record(stream)
+        for (d, g, rot) in cells:
+            for direction in ("fwd", "inv"):
+                launch(d, g, rot, direction)
+                i += 1
+                ev[k][i].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
-    total = start.elapsed_time(end)
-    fwd = sum(e[0].elapsed_time(e[1]) for e in ev)
-    inv = sum(e[1].elapsed_time(e[2]) for e in ev)
-    return total, fwd, inv
+    per = {}
+    for k in range(steps):
+        i = 0
+        for (d, g, rot) in cells:
+            for direction in ("fwd", "inv"):
+                per.setdefault((d, g, rot, direction), []).append(
+                    ev[k][i].elapsed_time(ev[k][i + 1]))
+                i += 1
+    return start.elapsed_time(end), per
 
 
-def run_e2e(kvq, x, signs, rot, g, packed, scales, out, world, steps, chunks=24):
-    n, d = x.shape
-    xh = x.cpu().pin_memory()
-    oh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
-    # chunk bounds on 32-row multiples keep every slice 16-byte aligned
-    bounds = [((i * n) // chunks) // 32 * 32 for i in range(chunks)] + [n]
+def cell_record(d, g, rot, direction, ms_list, n, peak):
+    best, med = min(ms_list), statistics.median(ms_list)
+    algo = n * fwd_bytes(d, g)
+    return {"cell": cell_name(d, g, rot, direction), "d": d, "group": g, "rot": ROTS[rot][1],
+            "dir": direction, "us_best": 1e3 * best, "us_median": 1e3 * med,
+            "algo_bytes": algo, "algo_gbs_median": algo / (med * 1e-3) / 1e9,
+            "frac_median": algo / (med * 1e-3) / 1e9 / peak,
+            "frac_best": algo / (best * 1e-3) / 1e9 / peak,
+            "fp16_gbs_median": n * d * 2 / (med * 1e-3) / 1e9,
+            "vec_per_s_median": n / (med * 1e-3)}
+
+
+def run_e2e(kvq, S, world, steps, chunks=8):
+    """The sweep through the public API with host buffers: every step copies
+    each d's inputs in from pinned host memory (chunked) and every cell's
+    output back; copies and kernels of consecutive chunks overlap on three
+    streams.  Same metric as the device-timed value."""
+    cells = [(g, rot) for g in (32, None) for rot, _ in ROTS]
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(chunks)]
-    ev_run = [torch.cuda.Event() for _ in range(chunks)]
-    ev_out = [torch.cuda.Event() for _ in range(chunks)]
+    nmax = max(T.n * T.d for T in S.values())
+    oh_all = torch.empty(nmax, dtype=torch.float16, pin_memory=True)
+    plan = {}
+    for d, T in S.items():
+        xh = torch.empty(T.x.shape, dtype=torch.float16, pin_memory=True)
+        xh.copy_(T.x)
+        bounds = [((i * T.n) // chunks) // 32 * 32 for i in range(chunks)] + [T.n]
+        plan[d] = (xh, oh_all[: T.n * d].view(T.n, d), bounds,
+                   [torch.cuda.Event() for _ in range(chunks)],  # input chunk landed
+                   [torch.cuda.Event() for _ in range(chunks)],  # input chunk free again
+                   [torch.cuda.Event() for _ in range(chunks)],  # kernels of the chunk done
+                   [torch.cuda.Event() for _ in range(chunks)])  # output chunk copied out
 
     def one_pass():
-        for c in range(chunks):
-            a, b = bounds[c], bounds[c + 1]
-            with torch.cuda.stream(s_in):
-                s_in.wait_event(ev_run[c])  # previous pass done reading x[a:b]
-                x[a:b].copy_(xh[a:b], non_blocking=True)
-                ev_in[c].record(s_in)
-            s_run.wait_event(ev_in[c])
-            s_run.wait_event(ev_out[c])  # previous pass done copying out[a:b]
-            kvq.kvq_rot_quant_fwd(x[a:b], signs, rot, g, packed[a:b], scales[a:b], s_run)
-            kvq.kvq_dequant_rot_inv(packed[a:b], scales[a:b], signs, rot, g, out[a:b], s_run)
-            ev_run[c].record(s_run)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_run[c])
-                oh[a:b].copy_(out[a:b], non_blocking=True)
-                ev_out[c].record(s_out)
+        for d, T in S.items():
+            xh, oh, bounds, ev_in, ev_free, ev_run, ev_out = plan[d]
+            for c in range(chunks):
+                a, b = bounds[c], bounds[c + 1]
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(ev_free[c])
+                    T.x[a:b].copy_(xh[a:b], non_blocking=True)
+                    ev_in[c].record(s_in)
+                s_run.wait_event(ev_in[c])
+                for i, (g, rot) in enumerate(cells):
+                    g = d if g is None else g
+                    kvq.kvq_rot_quant_fwd(T.x[a:b], T.signs, rot, g, T.packed[a:b],
+                                          T.scales[g][a:b], s_run)
+                    if i == len(cells) - 1:
+                        ev_free[c].record(s_run)
+                    s_run.wait_event(ev_out[c])  # previous cell's output chunk copied
+                    kvq.kvq_dequant_rot_inv(T.packed[a:b], T.scales[g][a:b], T.signs, rot, g,
+                                            T.out[a:b], s_run)
+                    ev_run[c].record(s_run)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(ev_run[c])
+                        oh[a:b].copy_(T.out[a:b], non_blocking=True)
+                        ev_out[c].record(s_out)
 
-    e2e_steps = max(3, min(steps, 10))
-    for _ in range(2):
-        one_pass()
+    e2e_steps = max(2, min(steps, 3))
+    one_pass()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -330,20 +475,270 @@ def run_e2e(kvq, x, signs, rot, g, packed, scales, out, world, steps, chunks=24)
         cur.wait_stream(st)
     e1.record(cur)
     torch.cuda.synchronize()
-    if not torch.equal(oh[: bounds[1]], out[: bounds[1]].cpu()):
+    last = S[SWEEP_D[-1]]
+    if not torch.equal(plan[last.d][1], last.out.cpu()):
         raise RuntimeError("end-to-end output differs from the device result")
     e2e_ms = allreduce_max(e0.elapsed_time(e1), world)
-    fp16_bytes_step = 2 * n * d * 2
-    return {"value": world * e2e_steps * fp16_bytes_step / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
-            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 2),
-            "chunks": chunks, "gpu_launches_per_step": 2 * chunks}
+    n_by_d = {d: T.n for d, T in S.items()}
+    fp16_in = sum(T.n * T.d * 2 for T in S.values())
+    return {"value": world * e2e_steps * sweep_fp16_bytes_per_step(n_by_d) / (e2e_ms * 1e-3) / 1e9,
+            "unit": UNIT, "h2d_bytes_per_step": int(fp16_in),
+            "d2h_bytes_per_step": int(len(cells) * fp16_in), "chunks_per_d": chunks,
+            "steps": e2e_steps, "gpu_launches_per_step": 2 * len(cells) * chunks * len(S)}
+
+
+# ----------------------------------------------------- CPU oracle legs ---
+
+def oracle_cell(O, xs, signs, rot, g):
+    """Oracle forward + inverse of the rows xs; returns (codes, scales, s)."""
+    t0 = time.perf_counter()
+    p, sc = O.rot_quant_fwd(xs, signs, rot, g)
+    O.dequant_rot_inv(p, sc, signs, rot, g)
+    return p, sc, time.perf_counter() - t0
+
+
+def flip_record(O, xs, signs, rot, g, p_ref, s_ref, p_gpu):
+    """Codes that differ between the GPU and the oracle, and how many of
+    them are not within 1e-4 of a rounding tie (must be 0)."""
+    q_ref = O.unpack_nibbles(p_ref)
+    q_gpu = O.unpack_nibbles(p_gpu)
+    bad = q_ref != q_gpu
+    n_bad = int(bad.sum())
+    not_tie = 0
+    if n_bad:
+        y = O.rotated_values(xs, signs, rot)
+        dist = O.near_tie_distance(y, s_ref, g)
+        not_tie = int((dist[bad] >= 1e-4).sum())
+    return {"codes": int(q_ref.size), "flips": n_bad, "flips_not_near_tie": not_tie}
+
+
+def cpu_legs(kvq, S, dev, peak_unused=None):
+    """The oracle on the host cores: (1) a sample of every sweep cell (the
+    cpu_baseline value, same weighting as the device step), (2) configs 1
+    and 3 and the config-4 decode step at position 256 on their full
+    tensors, (3) a sample of config 2; near-tie flip counts against the GPU
+    codes for each."""
+    import oracle.kvq_oracle as O
+    per_step_bytes, total_s, flips = 0, 0.0, {}
+    rows_per_d = {64: 16384, 128: 16384, 256: 8192}
+    for d, T in S.items():
+        idx = torch.from_numpy(W.sample_rows(T.n, rows_per_d[d], seed=7 + d)).to(dev)
+        xg = T.x[idx].contiguous()
+        xs = xg.cpu().numpy()
+        signs = W.make_signs(d)
+        for g in sweep_groups(d):
+            for rot, rname in ROTS:
+                p_gpu, _ = kvq.kvq_rot_quant_fwd(xg, T.signs, rot, g)
+                p, sc, dt = oracle_cell(O, xs, signs, rot, g)
+                total_s += dt
+                per_step_bytes += 2 * len(xs) * d * 2
+                flips[f"5 sweep d={d} g={g} {rname}"] = flip_record(
+                    O, xs, signs, rot, g, p, sc, p_gpu.cpu().numpy())
+    value = per_step_bytes / total_s / 1e9
+    sample = ", ".join(f"d={d}: {rows_per_d[d]} sampled rows" for d in S) + \
+        " of the sweep tensors, forward + inverse for every (g, rotation)"
+
+    per_config = {}
+    for i in (1, 3):
+        shape = W.config(i)
+        x = W.make_kv(shape)
+        xs = x.numpy()
+        xg = x.to(dev)
+        d, g = shape.d, shape.group
+        signs = W.make_signs(d)
+        sd = torch.from_numpy(signs).to(dev)
+        for rot, rname in ROTS:
+            p_gpu, _ = kvq.kvq_rot_quant_fwd(xg, sd, rot, g)
+            p, sc, dt = oracle_cell(O, xs, signs, rot, g)
+            per_config[f"{i} {shape.name} {rname}"] = {
+                "vectors": len(xs), "seconds": dt, "gbs": 2 * len(xs) * d * 2 / dt / 1e9}
+            flips[f"{i} {shape.name} {rname}"] = flip_record(O, xs, signs, rot, g, p, sc,
+                                                             p_gpu.cpu().numpy())
+    # config 4: one 26-layer decode step at position 256 (52 heads x 257 rows)
+    shape = W.scaled(W.config(4), tokens=257)
+    seq = W.make_decode_sequence(shape)  # [52, 257, 256]
+    d, g, pos = 256, 256, 256
+    signs = W.make_signs(d)
+    sd = torch.from_numpy(signs).to(dev)
+    for rot, rname in ROTS:
+        sq = seq.to(dev)
+        pk, sk = kvq.kvq_rot_quant_fwd(sq[:, :pos].reshape(-1, d).contiguous(), sd, rot, g)
+        packed = torch.zeros((52, pos + 1, d // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((52, pos + 1, 1), dtype=torch.float32, device=dev)
+        packed[:, :pos] = pk.reshape(52, pos, -1)
+        scales[:, :pos] = sk.reshape(52, pos, -1)
+        kvq.kvq_decode_step(sq[:, pos].contiguous(), packed, scales, pos, sd, rot, g)
+        xs = seq.reshape(-1, d).numpy()
+        p, sc, dt = oracle_cell(O, xs, signs, rot, g)
+        per_config[f"4 gemma3-1b decode step pos 256 {rname}"] = {
+            "vectors": len(xs), "seconds": dt, "gbs": 2 * len(xs) * d * 2 / dt / 1e9}
+        flips[f"4 gemma3-1b decode step pos 256 {rname}"] = flip_record(
+            O, xs, signs, rot, g, p, sc, packed.reshape(-1, d // 2).cpu().numpy())
+    # config 2: a sample of the SmolLM2-1.7B-shaped cache (same recipe, 4 heads)
+    shape = W.scaled(W.config(2), layers=1, heads=4)
+    x = W.make_kv(shape)
+    xs = x.numpy()
+    d, g = shape.d, shape.group
+    signs = W.make_signs(d)
+    sd = torch.from_numpy(signs).to(dev)
+    for rot, rname in ROTS:
+        p_gpu, _ = kvq.kvq_rot_quant_fwd(x.to(dev), sd, rot, g)
+        p, sc, dt = oracle_cell(O, xs, signs, rot, g)
+        per_config[f"2 {shape.name} sample {rname}"] = {
+            "vectors": len(xs), "seconds": dt, "gbs": 2 * len(xs) * d * 2 / dt / 1e9}
+        flips[f"2 {shape.name} sample {rname}"] = flip_record(O, xs, signs, rot, g, p, sc,
+                                                             p_gpu.cpu().numpy())
+    return ({"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+             "sample": sample, "seconds": total_s, "per_config": per_config},
+            flips)
+
+
+# -------------------------------------------------- other measurements ---
+
+def time_pair(kvq, x, packed, scales, out, signs, rot, g, steps, warmup):
+    """Per-launch device times (ms lists) of forward and inverse."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
+        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record(stream)
+        kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, stream)
+        ev[k][1].record(stream)
+        kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, stream)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    return ([e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev])
+
+
+def run_smollm2_cache(kvq, dev, peak, steps):
+    """Config 2 (SmolLM2-1.7B-shaped cache, d = g = 64): forward + inverse
+    of the whole cache per rotation."""
+    shape = W.config(2)
+    d, g = shape.d, shape.group
+    x = W.make_kv(shape, device=dev)
+    n = x.shape[0]
+    signs = torch.from_numpy(W.make_signs(d)).to(dev)
+    packed = torch.empty((n, d // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, d // g), dtype=torch.float32, device=dev)
+    out = torch.empty_like(x)
+    res = []
+    for rot, rname in ROTS:
+        f, i = time_pair(kvq, x, packed, scales, out, signs, rot, g, steps, 3)
+        for direction, ms in (("fwd", f), ("inv", i)):
+            rec = cell_record(d, g, rot, direction, ms, n, peak)
+            rec["cell"] = rec["cell"] + " (" + shape.name + ")"
+            res.append(rec)
+    del x, packed, scales, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode_latency(kvq, dev, peak, positions=(256, 1024, 2048, 4095), eager=False):
+    """Config 4 (Gemma-3-1B shape: 26 layers x K,V, d = g = 256): one decode
+    step = 26 kvq_decode_step calls (K and V of a layer as 2 heads), timed as
+    a CUDA graph at each position; the HBM bytes the step must move and the
+    time they take at the measured peak."""
+    shape = W.config(4)
+    d, g, L = 256, 256, 26
+    seq = W.make_decode_sequence(shape, device=dev)  # [52, 4096, 256]
+    signs = torch.from_numpy(W.make_signs(d)).to(dev)
+    cap = 4096
+    res = []
+    for rot, rname in ROTS:
+        packed = torch.zeros((2 * L, cap, d // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((2 * L, cap, 1), dtype=torch.float32, device=dev)
+        p, s = kvq.kvq_rot_quant_fwd(seq.reshape(-1, d), signs, rot, g)
+        packed.copy_(p.reshape(2 * L, cap, -1))
+        scales.copy_(s.reshape(2 * L, cap, -1))
+        for pos in positions:
+            outs = [torch.empty((2, pos + 1, d), dtype=torch.float16, device=dev)
+                    for _ in range(L)]
+            xs = [seq[2 * l:2 * l + 2, pos].contiguous() for l in range(L)]
+
+            def step():
+                for l in range(L):
+                    kvq.kvq_decode_step(xs[l], packed[2 * l:2 * l + 2], scales[2 * l:2 * l + 2],
+                                        pos, signs, rot, g, outs[l])
+            rec = {"rot": rname, "pos": pos}
+            if eager:
+                for _ in range(3):
+                    step()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(20):
+                    step()
+                e1.record()
+                torch.cuda.synchronize()
+                rec["eager_us_per_step"] = 1e3 * e0.elapsed_time(e1) / 20
+            rec["graph_us_per_step"] = graph_time_us(step)
+            # per head: new token in (2d) + its codes/scale out + pos+1 rows of
+            # codes/scales in and fp16 out (the new row's codes come from registers)
+            byts = L * 2 * ((pos + 1) * fwd_bytes(d, g) + 2 * d)
+            rec["algo_bytes_per_step"] = byts
+            rec["ideal_us"] = byts / (peak * 1e9) * 1e6
+            rec["frac"] = rec["ideal_us"] / rec["graph_us_per_step"]
+            res.append(rec)
+            del outs
+        del packed, scales
+    torch.cuda.empty_cache()
+    return res, seq, signs
+
+
+# ------------------------------------------------------------------ main ---
+
+def run_reference(args, world, rank):
+    """The CPU oracle, as it stands, on a bounded sample of the same sweep:
+    every step runs forward + inverse of `rows` vectors per (d, g, rotation)
+    cell, drawn from smaller tensors of the same recipe."""
+    if rank != 0:
+        return
+    import oracle.kvq_oracle as O
+    rows = 4096
+    data = {}
+    for d in SWEEP_D:
+        shape = W.scaled(W.config(5, d=d, group=32), heads=1)  # 16384 vectors of the recipe
+        data[d] = (W.make_kv(shape).numpy(), W.make_signs(d))
+    times, step_bytes = [], 0
+    for k in range(args.warmup + args.steps):
+        t = 0.0
+        step_bytes = 0
+        for d, g, rot in sweep_cells():
+            x, signs = data[d]
+            part = x[(k * rows) % len(x):][:rows]
+            _, _, dt = oracle_cell(O, part, signs, rot, g)
+            t += dt
+            step_bytes += 2 * len(part) * d * 2
+        if k >= args.warmup:
+            times.append(t)
+    total = sum(times)
+    value = step_bytes * len(times) / total / 1e9
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc() + f" (CPU oracle: {rows} vectors per cell "
+                                                 "per step)",
+                   "rows_per_cell_per_step": rows, "d": list(SWEEP_D), "group": "32, d",
+                   "rot": "srft, srht"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} vectors per (d, g, rotation) cell per step, drawn "
+                                   "from 16,384-vector tensors of the sweep recipe"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--suite", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -361,11 +756,13 @@ def main():
     ap.add_argument("--attn-nq", type=int, default=1)
     ap.add_argument("--decode-pos", type=int, default=0,
                     help="with --profile: run --reps 26-layer decode steps at this position")
-    args = ap.parse_args()
+    argv = sys.argv[1:]
+    args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     if args.profile:
         run_profile_case(args)
         return
+    maybe_relaunch(args, argv)
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, world, rank)
@@ -377,78 +774,62 @@ def main():
     from rotated_int4_kv_kvq_b200 import kvq
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    shape = headline_shape()
-    d, g, rot = shape.d, shape.group, kvq.SRFT
-    x = W.make_kv(shape, device=dev, seed=shape.seed + 1000 * rank)
-    n = x.shape[0]
-    signs = torch.from_numpy(W.make_signs(d)).to(dev)
-    packed = torch.empty((n, d // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((n, d // g), dtype=torch.float32, device=dev)
-    out = torch.empty_like(x)
+    peak, peak_kind = hbm_peak()
+    S = {d: SweepData(d, dev, seed_offset=1000 * rank) for d in SWEEP_D}
+    n_by_d = {d: T.n for d, T in S.items()}
 
-    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
-                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
-                           else local)
+    sampler = make_sampler(dev)
     sampler.start()
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
-    total_ms, fwd_ms, inv_ms = time_kernels(kvq, x, packed, scales, out, signs, rot, g,
-                                            args.steps, args.warmup, sampler)
+    total_ms, per = time_sweep(kvq, S, args.steps, args.warmup, sampler)
     barrier(world)
     sampler.stop()
     status = kvq.kvq_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status}")
     total_ms = allreduce_max(total_ms, world)
+    value = world * args.steps * sweep_fp16_bytes_per_step(n_by_d) / (total_ms * 1e-3) / 1e9
 
-    fp16_bytes_step = 2 * n * d * 2
-    value = world * args.steps * fp16_bytes_step / (total_ms * 1e-3) / 1e9
-    peak, peak_kind = hbm_peak()
-    algo = n * fwd_bytes(d, g)
-    dom, dom_ms = ("kvq_fwd_kernel", fwd_ms) if fwd_ms >= inv_ms else ("kvq_inv_kernel", inv_ms)
-    achieved = algo / (dom_ms * 1e-3 / args.steps) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(dom),
-                "kernel": dom, "peak_kind": peak_kind,
-                "algorithmic_bytes_per_launch": algo}
+    cells = [cell_record(d, g, rot, direction, per[(d, g, rot, direction)], n_by_d[d], peak)
+             for (d, g, rot) in sweep_cells() for direction in ("fwd", "inv")]
+    worst = min(cells, key=lambda c: c["frac_median"])
+    roofline = {"bound": "hbm", "achieved": worst["algo_gbs_median"], "peak": peak,
+                "unit": "GB/s", "frac": worst["frac_median"],
+                "traffic": recorded_traffic(worst["cell"]), "kernel": worst["cell"],
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": worst["algo_bytes"],
+                "launch_us_median": worst["us_median"]}
+    busiest = max(cells, key=lambda c: c["us_median"])
     detail = {
-        "fwd_us": 1e3 * fwd_ms / args.steps, "inv_us": 1e3 * inv_ms / args.steps,
-        "fwd_algo_gbs": algo / (fwd_ms * 1e-3 / args.steps) / 1e9,
-        "inv_algo_gbs": algo / (inv_ms * 1e-3 / args.steps) / 1e9,
-        "n_vec": n,
+        "sweep": cells,
+        "sweep_min_frac": worst["frac_median"],
+        "sweep_cells_below_0.70": [c["cell"] for c in cells if c["frac_median"] < 0.70],
+        "dominant_cell": busiest["cell"],
+        "vec_per_s": world * args.steps * sum(2 * n_by_d[d] for (d, g, rot) in sweep_cells())
+        / (total_ms * 1e-3),
+        "kernel_source_hash": kernel_source_hash(),
     }
-    detail["fwd_frac"] = detail["fwd_algo_gbs"] / peak
-    detail["inv_frac"] = detail["inv_algo_gbs"] / peak
-    # vectors per second: each direction alone, and through both per step
-    detail["fwd_vec_per_s"] = n / (fwd_ms * 1e-3 / args.steps)
-    detail["inv_vec_per_s"] = n / (inv_ms * 1e-3 / args.steps)
-    detail["vec_per_s"] = world * args.steps * n / (total_ms * 1e-3)
-    # SRHT control on the same cache (context)
-    t2, f2, i2 = time_kernels(kvq, x, packed, scales, out, signs, kvq.SRHT, g,
-                              max(10, args.steps // 4), 3)
-    k2 = max(10, args.steps // 4)
-    detail["srht_fwd_algo_gbs"] = algo / (f2 * 1e-3 / k2) / 1e9
-    detail["srht_inv_algo_gbs"] = algo / (i2 * 1e-3 / k2) / 1e9
-    detail["srht_value_gbs"] = k2 * fp16_bytes_step / (t2 * 1e-3) / 1e9
 
-    # end to end through the public API with host buffers: the cache streams
-    # in chunks; host->device copy, forward+inverse and device->host copy of
-    # consecutive chunks run on three streams and overlap.
-    e2e = run_e2e(kvq, x, signs, rot, g, packed, scales, out, world, args.steps)
+    e2e = run_e2e(kvq, S, world, args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        idx = W.sample_rows(n, 1 << 18, seed=7)
-        xs = x[torch.from_numpy(idx).to(dev)].cpu().numpy()
-        v, done, el = oracle_sample_gbs(xs, W.make_signs(d), 0, g, min_seconds=12.0)
-        cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{done} vectors (fwd+inv) drawn from {len(idx)} sampled rows of the "
-                         f"cache, {el:.1f} s"}
+        cpu, flips = cpu_legs(kvq, S, dev)
+        detail["near_tie_flips"] = flips
+    del S
+    torch.cuda.empty_cache()
+
+    if rank == 0:
+        detail["smollm2_1.7b_cache"] = run_smollm2_cache(kvq, dev, peak, args.steps)
+        detail["gemma3_1b_decode_step"], seq, signs = run_decode_latency(kvq, dev, peak)
+        detail["gemma3_1b_decode_step_windowed"] = run_window_suite(kvq, dev, seq, signs, peak)
+        del seq
+        torch.cuda.empty_cache()
 
     suite = None
     if args.suite and rank == 0:
-        suite_clock = ClockSampler(sampler.gpu)
+        suite_clock = make_sampler(dev)
         suite_clock.start()
         suite = run_suite(kvq, dev)
         suite_clock.stop()
@@ -463,11 +844,14 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": workload_desc(shape), "n_vec": n, "d": d, "group": g,
-                       "rot": "srft", "l2": "inputs larger than L2 (805 MB fp16 per pass), no flush",
+            "config": {"workload": workload_desc(), "n_vec_per_launch": n_by_d[64],
+                       "d": list(SWEEP_D), "group": "32, d", "rot": "srft, srht",
+                       "launches_per_step": 2 * len(sweep_cells()),
+                       "l2": "inputs larger than L2 (1.07-4.29 GB of fp16 per launch), no flush",
                        "parallelism": f"independent shards x{world} (no collective)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 2 * args.steps, "clocks": clocks, "detail": detail,
+            "gpu_launches": 2 * len(sweep_cells()) * args.steps, "clocks": clocks,
+            "detail": detail,
             "hbm_frac_of_nominal_8tbs": roofline["achieved"] / 8000.0,
         }
         print(json.dumps(line), flush=True)
@@ -554,135 +938,76 @@ def run_profile_decode(kvq, dev, args):
 
 
 def run_suite(kvq, dev):
-    """Large-batch sweep (every d, group, rotation, direction) and the
-    Gemma-3-1B decode-step latency."""
-    res = {"sweep": [], "decode": []}
+    """Measurements beyond the JSON line: other code widths and the lambda
+    hook on the sweep workload (g = d, SRFT), the eager decode step, and the
+    int4-reading attention."""
+    res = {}
     peak, _ = hbm_peak()
-    for d in (64, 128, 256):
-        for g in (32, d):
-            shape = W.config(5, d=d, group=g)
-            x = W.make_kv(shape, device=dev)
-            n = x.shape[0]
-            signs = torch.from_numpy(W.make_signs(d)).to(dev)
-            packed = torch.empty((n, d // 2), dtype=torch.uint8, device=dev)
-            scales = torch.empty((n, d // g), dtype=torch.float32, device=dev)
-            out = torch.empty_like(x)
-            algo = n * fwd_bytes(d, g)
-            for rot in (kvq.SRFT, kvq.SRHT):
-                # median of three timed rounds (single rounds move by a few
-                # percent between boxes and runs)
-                steps = 20
-                rounds = [time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 3)
-                          for _ in range(3)]
-                f = statistics.median(r[1] for r in rounds)
-                i = statistics.median(r[2] for r in rounds)
-                for name, ms in (("fwd", f), ("inv", i)):
-                    us = 1e3 * ms / steps
-                    res["sweep"].append({
-                        "d": d, "group": g, "rot": "srft" if rot == 0 else "srht", "dir": name,
-                        "us": us, "algo_gbs": algo / (us * 1e-6) / 1e9,
-                        "fp16_gbs": n * d * 2 / (us * 1e-6) / 1e9,
-                        "vec_per_s": n / (us * 1e-6), "frac": algo / (us * 1e-6) / 1e9 / peak})
-                if g == d and rot == kvq.SRFT:  # other code widths on the same workload
-                    for bits in ((3, 6, 8) if d >= 128 else (6, 8)):
-                        pb = torch.empty((n, d * bits // 8), dtype=torch.uint8, device=dev)
-                        ab = n * (2 * d + d * bits // 8 + 4 * (d // g))
-                        for _ in range(3):
-                            kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
-                            kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
-                        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                        tf = ti = 0.0
-                        for _ in range(steps):
-                            e[0].record()
-                            kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
-                            e[1].record()
-                            kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
-                            e[2].record()
-                            torch.cuda.synchronize()
-                            tf += e[0].elapsed_time(e[1])
-                            ti += e[1].elapsed_time(e[2])
-                        for name, ms in (("fwd", tf), ("inv", ti)):
-                            us = 1e3 * ms / steps
-                            res.setdefault("bits", []).append({
-                                "d": d, "group": g, "rot": "srft", "bits": bits, "dir": name,
-                                "us": us, "algo_gbs": ab / (us * 1e-6) / 1e9,
-                                "frac": ab / (us * 1e-6) / 1e9 / peak})
-                        del pb
-                if g == d:  # the per-channel lambda hook on the same workload
-                    lam = torch.exp(0.5 * torch.randn(d, generator=torch.Generator().manual_seed(d)))
-                    lam = lam.to(dev)
-                    tot, f, i = time_kernels(kvq, x, packed, scales, out, signs, rot, g, steps, 3,
-                                             lam=lam)
-                    for name, ms in (("fwd", f), ("inv", i)):
+    steps = 20
+    for d in SWEEP_D:
+        g = d
+        shape = W.config(5, d=d, group=g)
+        x = W.make_kv(shape, device=dev)
+        n = x.shape[0]
+        signs = torch.from_numpy(W.make_signs(d)).to(dev)
+        packed = torch.empty((n, d // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((n, d // g), dtype=torch.float32, device=dev)
+        out = torch.empty_like(x)
+        algo = n * fwd_bytes(d, g)
+        for rot, rname in ROTS:
+            if rot == 0:  # other code widths on the same workload
+                for bits in ((3, 6, 8) if d >= 128 else (6, 8)):
+                    pb = torch.empty((n, d * bits // 8), dtype=torch.uint8, device=dev)
+                    ab = n * (2 * d + d * bits // 8 + 4 * (d // g))
+                    for _ in range(3):
+                        kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
+                        kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
+                    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    tf = ti = 0.0
+                    for _ in range(steps):
+                        e[0].record()
+                        kvq.kvq_rot_quant_fwd_bits(x, signs, rot, g, bits, pb, scales)
+                        e[1].record()
+                        kvq.kvq_dequant_rot_inv_bits(pb, scales, signs, rot, g, bits, out)
+                        e[2].record()
+                        torch.cuda.synchronize()
+                        tf += e[0].elapsed_time(e[1])
+                        ti += e[1].elapsed_time(e[2])
+                    for name, ms in (("fwd", tf), ("inv", ti)):
                         us = 1e3 * ms / steps
-                        res.setdefault("lambda", []).append({
-                            "d": d, "group": g, "rot": "srft" if rot == 0 else "srht",
-                            "dir": name, "us": us, "algo_gbs": algo / (us * 1e-6) / 1e9,
-                            "frac": algo / (us * 1e-6) / 1e9 / peak})
-            del x, packed, scales, out
-            torch.cuda.empty_cache()
-    # decode: 26 layers x (K, V) x d=256, g=256; one call per layer (2 heads)
-    shape = W.config(4)
-    d, g, L = 256, 256, 26
-    seq = W.make_decode_sequence(shape, device=dev)  # [52, 4096, 256]
-    signs = torch.from_numpy(W.make_signs(d)).to(dev)
-    cap = 4096
-    for rot in (kvq.SRFT, kvq.SRHT):
-        packed = torch.zeros((2 * L, cap, d // 2), dtype=torch.uint8, device=dev)
-        scales = torch.zeros((2 * L, cap, 1), dtype=torch.float32, device=dev)
-        p, s = kvq.kvq_rot_quant_fwd(seq.reshape(-1, d), signs, rot, g)
-        packed.copy_(p.reshape(2 * L, cap, -1))
-        scales.copy_(s.reshape(2 * L, cap, -1))
-        for pos in (256, 1024, 2048, 4095):
-            outs = [torch.empty((2, pos + 1, d), dtype=torch.float16, device=dev)
-                    for _ in range(L)]
-            xs = [seq[2 * l:2 * l + 2, pos].contiguous() for l in range(L)]
-
-            def step():
-                for l in range(L):
-                    kvq.kvq_decode_step(xs[l], packed[2 * l:2 * l + 2], scales[2 * l:2 * l + 2],
-                                        pos, signs, rot, g, outs[l])
+                        res.setdefault("bits", []).append({
+                            "d": d, "group": g, "rot": rname, "bits": bits, "dir": name,
+                            "us": us, "algo_gbs": ab / (us * 1e-6) / 1e9,
+                            "frac": ab / (us * 1e-6) / 1e9 / peak})
+                    del pb
+            # the per-channel lambda hook on the same workload
+            lam = torch.exp(0.5 * torch.randn(d, generator=torch.Generator().manual_seed(d)))
+            lam = lam.to(dev)
             for _ in range(3):
-                step()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = 20
-            e0.record()
-            for _ in range(reps):
-                step()
-            e1.record()
-            torch.cuda.synchronize()
-            eager_us = 1e3 * e0.elapsed_time(e1) / reps
-            graph_us = None
-            try:
-                gr = torch.cuda.CUDAGraph()
-                s2 = torch.cuda.Stream()
-                s2.wait_stream(torch.cuda.current_stream())
-                with torch.cuda.stream(s2):
-                    step()
-                torch.cuda.current_stream().wait_stream(s2)
-                with torch.cuda.graph(gr):
-                    step()
-                for _ in range(3):
-                    gr.replay()
+                kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, lam=lam)
+                kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, lam=lam)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            tf = ti = 0.0
+            for _ in range(steps):
+                e[0].record()
+                kvq.kvq_rot_quant_fwd(x, signs, rot, g, packed, scales, lam=lam)
+                e[1].record()
+                kvq.kvq_dequant_rot_inv(packed, scales, signs, rot, g, out, lam=lam)
+                e[2].record()
                 torch.cuda.synchronize()
-                e0.record()
-                for _ in range(reps):
-                    gr.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                graph_us = 1e3 * e0.elapsed_time(e1) / reps
-                del gr
-            except Exception as ex:  # capture unsupported: report eager only
-                graph_us = f"capture failed: {ex}"
-            # per head: new token in (2d) + its codes/scale out + pos+1 rows of
-            # codes/scales in and fp16 out (the new row's codes come from registers)
-            byts = L * 2 * ((pos + 1) * fwd_bytes(d, g) + 2 * d)
-            res["decode"].append({"rot": "srft" if rot == 0 else "srht", "pos": pos,
-                                  "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
-                                  "algo_bytes_per_step": byts,
-                                  "ideal_us": byts / (peak * 1e9) * 1e6})
-    res["decode_windowed"] = run_window_suite(kvq, dev, seq, signs, peak)
+                tf += e[0].elapsed_time(e[1])
+                ti += e[1].elapsed_time(e[2])
+            for name, ms in (("fwd", tf), ("inv", ti)):
+                us = 1e3 * ms / steps
+                res.setdefault("lambda", []).append({
+                    "d": d, "group": g, "rot": rname, "dir": name, "us": us,
+                    "algo_gbs": algo / (us * 1e-6) / 1e9,
+                    "frac": algo / (us * 1e-6) / 1e9 / peak})
+        del x, packed, scales, out
+        torch.cuda.empty_cache()
+    res["decode"], seq, signs = run_decode_latency(kvq, dev, peak, eager=True)
+    del seq
+    torch.cuda.empty_cache()
     res["attention"] = run_attention_suite(kvq, dev, peak)
     return res
 

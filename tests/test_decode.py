@@ -126,3 +126,67 @@ def test_gemma_decode_steps(kvq):
                               out.reshape(-1, d).cpu().numpy(), flipped)
         torch.cuda.synchronize()
         assert kvq.kvq_device_status() == 0
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+def test_decode_52_heads_just_past_the_wide_limit(kvq, rot):
+    """52 heads in one call at pos 1260 (65,572 rows): the first position at
+    which a 52-head call leaves the one-warp-per-vector kernel."""
+    assert 52 * 1261 > WIDE_MAX_ROWS >= 52 * 1260
+    run_and_check(kvq, 256, 256, rot, heads=52, cap=1262, pos=1260, seed=11 + rot)
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+def test_gemma_decode_step_across_the_prefix_sweep(kvq, rot):
+    """Config 4 at the prefix lengths the step is measured at (pos 1024,
+    2048, 4095): the cache rows [0, pos) come from the forward call over the
+    token stream, then one 26-call decode step (K and V of a layer as two
+    heads) runs at pos.  Every layer's new row is checked against the oracle
+    (codes, scales, x_hat), and every output row of every layer against the
+    oracle inverse of the stored codes and scales."""
+    shape = W.config(4)
+    seq = W.make_decode_sequence(shape, device="cuda")  # [52, 4096, 256]
+    d, group, cap = 256, 256, 4096
+    signs_np = W.make_signs(d)
+    signs = torch.from_numpy(signs_np).cuda()
+    seq_np = seq.cpu().numpy()
+    flips = codes = 0
+    for pos in (1024, 2048, 4095):
+        packed = torch.zeros((52, cap, d // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((52, cap, 1), dtype=torch.float32, device="cuda")
+        p, s = kvq.kvq_rot_quant_fwd(seq[:, :pos].reshape(-1, d).contiguous(), signs, rot, group)
+        packed[:, :pos] = p.reshape(52, pos, -1)
+        scales[:, :pos] = s.reshape(52, pos, -1)
+        outs = []
+        for layer in range(26):
+            hs = slice(2 * layer, 2 * layer + 2)
+            outs.append(kvq.kvq_decode_step(seq[hs, pos].contiguous(), packed[hs], scales[hs],
+                                            pos, signs, rot, group))
+        torch.cuda.synchronize()
+        assert kvq.kvq_device_status() == 0
+        out = torch.cat(outs).cpu().numpy()  # [52, pos + 1, 256]
+        # the new row of every head against the oracle
+        x_new = seq_np[:, pos]
+        p_new = packed[:, pos].cpu().numpy()
+        s_new = scales[:, pos].cpu().numpy()
+        q, _, nf, _, flipped = check_fwd(x_new, signs_np, rot, group, p_new, s_new,
+                                         max_flip_fraction=None)
+        flips += nf
+        codes += q.size
+        check_inv(x_new, signs_np, rot, group, p_new, s_new, out[:, pos], flipped)
+        # every row of every head against the oracle inverse of the stored codes
+        rows_p = packed[:, : pos + 1].reshape(-1, d // 2).cpu().numpy()
+        rows_s = scales[:, : pos + 1].reshape(-1, 1).cpu().numpy()
+        ref_o = O.dequant_rotated_f64(rows_p, rows_s, signs_np, rot, group)
+        got = out.reshape(-1, d).astype(np.float64)
+        tol = 2e-3 * np.abs(ref_o).max(axis=1, keepdims=True) + 1e-6
+        assert np.all(np.abs(got - ref_o) <= tol)
+        # the cached codes themselves against the oracle's forward step
+        q, _, nf, _, _ = check_fwd(seq_np[:, :pos].reshape(-1, d), signs_np, rot, group,
+                                   rows_p.reshape(52, pos + 1, -1)[:, :pos].reshape(-1, d // 2),
+                                   rows_s.reshape(52, pos + 1, -1)[:, :pos].reshape(-1, 1),
+                                   max_flip_fraction=None)
+        flips += nf
+        codes += q.size
+        del packed, scales, outs
+    assert flips < 1e-4 * codes, f"{flips} near-tie flips of {codes} codes"
