@@ -29,6 +29,25 @@
 
 namespace kvq {
 
+// Test builds only: the forward kernel arms the mbarrier of this input tile
+// but issues no copy for it, so the wait on it runs out (with nothing in
+// flight) and the time-out path is exercised.  -1 (every product build):
+// every tile is loaded.
+#ifndef KVQ_TEST_SKIP_TILE
+#define KVQ_TEST_SKIP_TILE (-1)
+#endif
+
+// Round the SRFT join outputs with packed f32x2 multiply-adds (1) or one
+// scalar multiply-add per value (0).
+#ifndef KVQ_SRFT_QFMA2
+#define KVQ_SRFT_QFMA2 0
+#endif
+// Flip and widen the fp16 inputs with one mixed-precision multiply-add per
+// sample (1), or XOR the sign bits and widen (0).
+#ifndef KVQ_MIXED_CVT
+#define KVQ_MIXED_CVT 0
+#endif
+
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 
@@ -178,37 +197,47 @@ __device__ __forceinline__ uint32_t swq(int row, int c) {
   return uint32_t(row * P + ((c ^ (((row * P) >> 7) & (P / 16 - 1))) << 4));
 }
 
+// Sign-flipped fp16 word w (samples (lo, hi)) widened to an f32 pair.  With
+// KVQ_MIXED_CVT the sign table entry m holds fp16 +-1 pairs and one
+// mixed-precision multiply-add per sample flips and widens it; otherwise m
+// holds sign-bit masks XOR-ed into the word before a plain widening.
+__device__ __forceinline__ f2 signed_pair(uint32_t w, uint32_t m) {
+#if KVQ_MIXED_CVT
+  return half2_times_signs(w, m);
+#else
+  const float2 f = half2_bits_to_float2(w ^ m);
+  return mk2(f.x, f.y);
+#endif
+}
+
+// Thread t's words of the row, sign-flipped and widened to f32 pairs.
 template <class C>
 __device__ __forceinline__ void load_x(uint32_t tile, int row, int t, uint32_t mask,
-                                       uint32_t (&xw)[C::NW]) {
+                                       f2 (&u)[C::NW]) {
   if constexpr (!C::PAIR_RFFT) {
 #pragma unroll
     for (int c = 0; c < C::NW / 4; ++c) {
       const int gc = t * (C::NW / 4) + c;  // chunk of the row
       const uint4 v = lds128(tile + (gc / 8) * C::SLAB + sw128(row, gc % 8));
       const uint4 m = lds128(mask + c * 16);
-      xw[4 * c + 0] = v.x ^ m.x;
-      xw[4 * c + 1] = v.y ^ m.y;
-      xw[4 * c + 2] = v.z ^ m.z;
-      xw[4 * c + 3] = v.w ^ m.w;
+      u[4 * c + 0] = signed_pair(v.x, m.x);
+      u[4 * c + 1] = signed_pair(v.y, m.y);
+      u[4 * c + 2] = signed_pair(v.z, m.z);
+      u[4 * c + 3] = signed_pair(v.w, m.w);
     }
   } else {
     // Both threads of the pair read the whole row; thread t keeps fp16 half
     // t of every word, two words per result: (u_{4j+t}, u_{4j+2+t}).
     const uint32_t sel = t ? 0x7632u : 0x5410u;
 #pragma unroll
-    for (int c = 0; c < C::D / 8; ++c) {
-      const uint4 v = lds128(tile + (c / 8) * C::SLAB + sw128(row, c % 8));
-      xw[2 * c] = __byte_perm(v.x, v.y, sel);
-      xw[2 * c + 1] = __byte_perm(v.z, v.w, sel);
-    }
-#pragma unroll
-    for (int c = 0; c < C::NW / 4; ++c) {
+    for (int c = 0; c < C::D / 16; ++c) {
       const uint4 m = lds128(mask + c * 16);
-      xw[4 * c] ^= m.x;
-      xw[4 * c + 1] ^= m.y;
-      xw[4 * c + 2] ^= m.z;
-      xw[4 * c + 3] ^= m.w;
+      const uint4 v0 = lds128(tile + ((2 * c) / 8) * C::SLAB + sw128(row, (2 * c) % 8));
+      const uint4 v1 = lds128(tile + ((2 * c + 1) / 8) * C::SLAB + sw128(row, (2 * c + 1) % 8));
+      u[4 * c + 0] = signed_pair(__byte_perm(v0.x, v0.y, sel), m.x);
+      u[4 * c + 1] = signed_pair(__byte_perm(v0.z, v0.w, sel), m.y);
+      u[4 * c + 2] = signed_pair(__byte_perm(v1.x, v1.y, sel), m.z);
+      u[4 * c + 3] = signed_pair(__byte_perm(v1.z, v1.w, sel), m.w);
     }
   }
 }
@@ -381,32 +410,33 @@ __device__ __forceinline__ void pair_join_fwd(const f2 (&y)[C::D / 4], int t, f2
     const float ox = lo2(y[a]), oy = hi2(y[a]);
     const float rx = __shfl_xor_sync(kFull, lo2(y[H - a]), 1);
     const float ry = __shfl_xor_sync(kFull, hi2(y[H - a]), 1);
-    // thread 0 twiddles conj(received) = O_a, thread 1 its own V_a
-    const float tx = odd ? ox : rx, ty = odd ? oy : -ry;
+    // thread 0 twiddles conj(received) = O_a, thread 1 its own V_a times
+    // -i (W_d^{NR/2+a} = -i W_d^a), i.e. (Im V_a, -Re V_a): the same twiddle
+    // code then gives both threads their q / m
+    const float tx = odd ? oy : rx, ty = -(odd ? ox : ry);
     const float px = odd ? rx : ox, py = odd ? -ry : oy;  // E (thread 1: conj E)
-    float m, hx, hy;  // W_d^a t = m (hx, hy)
-    twiddle_tan<a, C::D>(tx, ty, m, hx, hy);
-    const float qx = odd ? hy : hx, qy = odd ? -hx : hy;  // q / m
+    float m, qx, qy;  // q = W_d^a t = m (qx, qy)
+    twiddle_tan<a, C::D>(tx, ty, m, qx, qy);
     if constexpr (a < H / 2) Y[a] = mk2(fmaf(m, qx, px), fmaf(m, qy, py));
     Y[H - a] = mk2(fmaf(-m, qx, px), fmaf(m, qy, -py));
   });
 }
 
 // Y: this thread's E rotated coordinates as P pairs (local order of the
-// layout), unnormalized: the true y is KAPPA * Y.  Input: sign-flipped fp16
-// words.
+// layout), unnormalized: the true y is KAPPA * Y.  Input: the sign-flipped
+// samples of load_x (consumed).
 // With LAM, the values are multiplied by the load-side lambda pairs at
 // `lam` (shared memory) first.
 template <class C, bool LAM = false>
-__device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f2 (&Y)[C::P],
+__device__ __forceinline__ void rotate_fwd(f2 (&u)[C::NW], int t, f2 (&Y)[C::P],
                                            uint32_t lam = 0) {
+  if constexpr (LAM) {
+#pragma unroll
+    for (int j = 0; j < C::NW; ++j) u[j] = mul2(u[j], lds_f2(lam + 8u * j));
+  }
   if constexpr (C::ROT == kRotSRHT) {
 #pragma unroll
-    for (int j = 0; j < C::NW; ++j) {
-      const float2 f = half2_bits_to_float2(xw[j]);
-      Y[j] = mk2(f.x, f.y);
-      if constexpr (LAM) Y[j] = mul2(Y[j], lds_f2(lam + 8u * j));
-    }
+    for (int j = 0; j < C::NW; ++j) Y[j] = u[j];
     fwht<C::P>(Y);
     if constexpr (C::TPV == 2) {
       // H_d = [[H, H], [H, -H]] across the pair, exchanging half the data.
@@ -429,13 +459,7 @@ __device__ __forceinline__ void rotate_fwd(const uint32_t (&xw)[C::NW], int t, f
   } else {
     // Each word is (even, odd) sample: one two-lane codelet transforms both
     // parity halves of this thread's E samples, the join makes their rfft.
-    f2 u[C::NW], y2[C::NW];
-#pragma unroll
-    for (int j = 0; j < C::NW; ++j) {
-      const float2 f = half2_bits_to_float2(xw[j]);
-      u[j] = mk2(f.x, f.y);
-      if constexpr (LAM) u[j] = mul2(u[j], lds_f2(lam + 8u * j));
-    }
+    f2 y2[C::NW];
     RFFT2<C::E / 2>::fwd(u, y2);
     if constexpr (C::TPV == 1) {
       join_lanes_fwd<C::E, C::D != 128>(y2, Y);
@@ -528,6 +552,14 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     if constexpr (LAM) v = mul2(v, lds_f2(lam + 8u * j));
     return float2_to_half2_bits(lo2(v), hi2(v));
   };
+  // With LAM, a warp barrier after every 8 converted words: shared-memory
+  // loads are not moved across it, so at most 8 lambda pairs are live at a
+  // time (loaded all at once, they pushed the register demand into spills).
+  auto fence = [&](int j) {
+    if constexpr (LAM) {
+      if (j % 8 == 7) __syncwarp();
+    }
+  };
   if constexpr (C::ROT == kRotSRHT) {
     if constexpr (C::TPV == 2) {
       // Inverse of rotate_fwd's pair step: from a = y_k, b = y_{k+d/2} of
@@ -548,7 +580,10 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     }
     fwht<C::P>(Y);
 #pragma unroll
-    for (int j = 0; j < C::NW; ++j) xw[j] = scaled(Y[j], j);
+    for (int j = 0; j < C::NW; ++j) {
+      xw[j] = scaled(Y[j], j);
+      fence(j);
+    }
   } else {
     f2 z[C::NW], x2[C::NW];
     if constexpr (C::TPV == 1) {
@@ -561,7 +596,10 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
     RFFT2<C::E / 2>::inv(z, x2);
     if constexpr (C::TPV == 1) {
 #pragma unroll
-      for (int n = 0; n < C::NW; ++n) xw[n] = scaled(x2[n], n);
+      for (int n = 0; n < C::NW; ++n) {
+        xw[n] = scaled(x2[n], n);
+        fence(n);
+      }
     } else {
       // Thread 0 holds the even samples e_m, thread 1 r_m = (-1)^m o_{m+NR/2}
       // (o: odd samples), as fp16 pairs P_i = (s_{2i}, s_{2i+1}).  Both keep
@@ -573,6 +611,7 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
       for (int i = 0; i < C::NW / 2; ++i) {
         const uint32_t own = scaled(x2[i], i);
         const uint32_t r = __shfl_xor_sync(kFull, scaled(x2[i + C::NW / 2], i + C::NW / 2), 1);
+        fence(2 * i + 1);
         xw[2 * i] = __byte_perm(own, r, se);
         xw[2 * i + 1] = __byte_perm(own, r, so);
       }
@@ -678,7 +717,7 @@ __device__ __forceinline__ void quantize(const f2 (&Y)[C::P], uint32_t (&qw)[C::
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const f2 v = Y[g * GP + 4 * w + i];
-        if constexpr (C::ROT == kRotSRFT) {  // scalar join outputs: no re-pairing
+        if constexpr (C::ROT == kRotSRFT && !KVQ_SRFT_QFMA2) {  // scalar join outputs
           f[2 * i] = __float_as_uint(__fmaf_rn(lo2(v), inv, kRoundMagic));
           f[2 * i + 1] = __float_as_uint(__fmaf_rn(hi2(v), inv, kRoundMagic));
         } else {
@@ -800,7 +839,9 @@ template <class C>
 __device__ __forceinline__ void fill_sign_masks(const int8_t* signs, uint32_t* s_mask) {
   for (int i = threadIdx.x; i < C::D / 2; i += blockDim.x) {
     const int t = i / C::NW, j = i % C::NW;
-    s_mask[i] = load_mask_word<C>(signs, t, j);
+    // load side: sign-bit masks, or fp16 +-1 pairs for the mixed-precision
+    // flip (0x3C00 = 1.0, 0xBC00 = -1.0)
+    s_mask[i] = load_mask_word<C>(signs, t, j) ^ (KVQ_MIXED_CVT ? 0x3C003C00u : 0u);
     s_mask[C::D / 2 + i] = store_mask_word<C>(signs, t, j);
   }
 }
@@ -907,9 +948,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
     const uint32_t bar = bars + 8u * s;
     const uint32_t dst = xbuf + uint32_t(s * C::XTILE);
     mbar_arrive_expect_tx(bar, C::XTILE);
+    if (KVQ_TEST_SKIP_TILE < 0 || tile != KVQ_TEST_SKIP_TILE) {
 #pragma unroll
-    for (int j = 0; j < C::D / 64; ++j)
-      tma_load_2d(dst + j * C::SLAB, &tmX, bar, 64 * j, int(tile * C::VPW));
+      for (int j = 0; j < C::D / 64; ++j)
+        tma_load_2d(dst + j * C::SLAB, &tmX, bar, 64 * j, int(tile * C::VPW));
+    }
     ++ring.issued;
   };
   if (lane == 0)
@@ -924,8 +967,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
       break;
     }
     ++ring.consumed;
-    uint32_t xw[C::NW];
-    load_x<C>(xbuf + uint32_t(s * C::XTILE), row, t, mask, xw);
+    f2 u[C::NW];
+    load_x<C>(xbuf + uint32_t(s * C::XTILE), row, t, mask, u);
     __syncwarp();
     if (lane == 0) {
       const int64_t nt = tile + int64_t(S_IN) * nw;
@@ -935,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
       }
     }
     f2 Y[C::P];
-    rotate_fwd<C, LAM>(xw, t, Y, lam);
+    rotate_fwd<C, LAM>(u, t, Y, lam);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
     quantize<C, G>(Y, qw, sc, t);
@@ -1126,10 +1169,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
       return;
     }
     new_phase ^= 1u;
-    uint32_t xw[C::NW];
-    load_x<C>(xin, row, t, mask, xw);
+    f2 u[C::NW];
+    load_x<C>(xin, row, t, mask, u);
     f2 Y[C::P];
-    rotate_fwd<C>(xw, t, Y);
+    rotate_fwd<C>(u, t, Y);
     uint32_t qw[C::NQ];
     float sc[Gr::NL];
     quantize<C, G>(Y, qw, sc, t);
@@ -1142,6 +1185,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         if (writes_scale<C, G>(t, lg)) p[global_group<C, G>(t, lg)] = sc[lg];
     }
     dequantize<C, G>(qw, sc, Y);
+    uint32_t xw[C::NW];
     rotate_inv<C>(Y, t, xw);
     store_x<C>(xout, row, t, mask_st, xw);
     fence_proxy_async_smem();

@@ -161,14 +161,23 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after ~2 s (or 2^26
-// polls).  Returns false on time-out; callers record the error and stop.
+// Limits of a bounded wait: wall time (ns) and number of polls.
+#ifndef KVQ_WAIT_LIMIT_NS
+#define KVQ_WAIT_LIMIT_NS 2000000000ull
+#endif
+#ifndef KVQ_WAIT_MAX_POLLS
+#define KVQ_WAIT_MAX_POLLS (1u << 26)
+#endif
+
+// Wait for phase `parity` of an mbarrier, giving up after KVQ_WAIT_LIMIT_NS
+// (~2 s) or KVQ_WAIT_MAX_POLLS polls.  Returns false on time-out; callers
+// record the error and stop.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1; it < (1u << 26); ++it) {
+  for (uint32_t it = 1; it < KVQ_WAIT_MAX_POLLS; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 0 && global_timer_ns() - t0 > 2000000000ull) return false;
+    if ((it & 1023u) == 0 && global_timer_ns() - t0 > KVQ_WAIT_LIMIT_NS) return false;
   }
   return false;
 }
@@ -309,6 +318,21 @@ __device__ __forceinline__ f2 mk2(float x, float y) {
   f2 r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(x), "f"(y));
   return r;
+}
+
+// The fp16 pair w times the fp16 pair m (+-1 each), widened to f32: one
+// mixed-precision multiply-add per half (f16 x f16 + f32 -> f32, exact for a
+// sign), adding -0 so that a -0 product stays -0.
+__device__ __forceinline__ f2 half2_times_signs(uint32_t w, uint32_t m) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 a0, a1, s0, s1;\n\t"
+      "mov.b32 {a0, a1}, %2;\n\t"
+      "mov.b32 {s0, s1}, %3;\n\t"
+      "fma.rn.f32.f16 %0, a0, s0, 0f80000000;\n\t"
+      "fma.rn.f32.f16 %1, a1, s1, 0f80000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w), "r"(m));
+  return mk2(lo, hi);
 }
 // An f2 from shared memory (8-byte aligned address).
 __device__ __forceinline__ f2 lds_f2(uint32_t a) {
