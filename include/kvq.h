@@ -65,6 +65,15 @@
 extern "C" {
 #endif
 
+/* The library is built with hidden symbol visibility: only the functions
+ * declared here are exported, so two builds loaded into one process (for
+ * instance a test build beside the product one) share no internal state. */
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *kvq_stream;
 
@@ -102,9 +111,9 @@ typedef enum {
  *   scales  [n_vec][d/g] fp32, 16-byte aligned (written)
  *   stream  CUDA stream
  */
-kvq_status kvq_rot_quant_fwd(const uint16_t *x, int64_t n_vec, int32_t d,
-                             int32_t group, const int8_t *signs, kvq_rot rot,
-                             uint8_t *packed, float *scales, kvq_stream stream);
+KVQ_API kvq_status kvq_rot_quant_fwd(const uint16_t *x, int64_t n_vec, int32_t d,
+                                     int32_t group, const int8_t *signs, kvq_rot rot,
+                                     uint8_t *packed, float *scales, kvq_stream stream);
 
 /*
  * Inverse step ("First, the 17%": dequantized and rotated back when
@@ -116,10 +125,10 @@ kvq_status kvq_rot_quant_fwd(const uint16_t *x, int64_t n_vec, int32_t d,
  *   out     [n_vec][d] fp16, 16-byte aligned (written): x_hat = D R^T (s q)
  *   other arguments as in kvq_rot_quant_fwd.
  */
-kvq_status kvq_dequant_rot_inv(const uint8_t *packed, const float *scales,
-                               int64_t n_vec, int32_t d, int32_t group,
-                               const int8_t *signs, kvq_rot rot, uint16_t *out,
-                               kvq_stream stream);
+KVQ_API kvq_status kvq_dequant_rot_inv(const uint8_t *packed, const float *scales,
+                                       int64_t n_vec, int32_t d, int32_t group,
+                                       const int8_t *signs, kvq_rot rot, uint16_t *out,
+                                       kvq_stream stream);
 
 /*
  * Forward and inverse steps with a per-channel factor lambda, the kernel
@@ -134,16 +143,16 @@ kvq_status kvq_dequant_rot_inv(const uint8_t *packed, const float *scales,
  *           non-zero (not checked on the device).  NULL -> KVQ_ERR_NULL.
  *   other arguments as in kvq_rot_quant_fwd / kvq_dequant_rot_inv.
  */
-kvq_status kvq_rot_quant_fwd_lambda(const uint16_t *x, int64_t n_vec, int32_t d,
-                                    int32_t group, const int8_t *signs,
-                                    const float *lambda, kvq_rot rot,
-                                    uint8_t *packed, float *scales,
-                                    kvq_stream stream);
-kvq_status kvq_dequant_rot_inv_lambda(const uint8_t *packed, const float *scales,
-                                      int64_t n_vec, int32_t d, int32_t group,
-                                      const int8_t *signs, const float *lambda,
-                                      kvq_rot rot, uint16_t *out,
-                                      kvq_stream stream);
+KVQ_API kvq_status kvq_rot_quant_fwd_lambda(const uint16_t *x, int64_t n_vec, int32_t d,
+                                            int32_t group, const int8_t *signs,
+                                            const float *lambda, kvq_rot rot,
+                                            uint8_t *packed, float *scales,
+                                            kvq_stream stream);
+KVQ_API kvq_status kvq_dequant_rot_inv_lambda(const uint8_t *packed, const float *scales,
+                                              int64_t n_vec, int32_t d, int32_t group,
+                                              const int8_t *signs, const float *lambda,
+                                              kvq_rot rot, uint16_t *out,
+                                              kvq_stream stream);
 
 /*
  * Forward and inverse steps with another code width b ("Quantization Speed
@@ -159,16 +168,16 @@ kvq_status kvq_dequant_rot_inv_lambda(const uint8_t *packed, const float *scales
  *   packed  [n_vec][d*bits/8] uint8, 16-byte aligned
  *   other arguments as in kvq_rot_quant_fwd / kvq_dequant_rot_inv.
  */
-kvq_status kvq_rot_quant_fwd_bits(const uint16_t *x, int64_t n_vec, int32_t d,
-                                  int32_t group, int32_t bits,
-                                  const int8_t *signs, kvq_rot rot,
-                                  uint8_t *packed, float *scales,
-                                  kvq_stream stream);
-kvq_status kvq_dequant_rot_inv_bits(const uint8_t *packed, const float *scales,
-                                    int64_t n_vec, int32_t d, int32_t group,
-                                    int32_t bits, const int8_t *signs,
-                                    kvq_rot rot, uint16_t *out,
-                                    kvq_stream stream);
+KVQ_API kvq_status kvq_rot_quant_fwd_bits(const uint16_t *x, int64_t n_vec, int32_t d,
+                                          int32_t group, int32_t bits,
+                                          const int8_t *signs, kvq_rot rot,
+                                          uint8_t *packed, float *scales,
+                                          kvq_stream stream);
+KVQ_API kvq_status kvq_dequant_rot_inv_bits(const uint8_t *packed, const float *scales,
+                                            int64_t n_vec, int32_t d, int32_t group,
+                                            int32_t bits, const int8_t *signs,
+                                            kvq_rot rot, uint16_t *out,
+                                            kvq_stream stream);
 
 /*
  * Decode step for one head-major cache, one launch ("A scene" and "First,
@@ -190,11 +199,11 @@ kvq_status kvq_dequant_rot_inv_bits(const uint8_t *packed, const float *scales,
  *   out     [n_heads][pos+1][d] fp16, 16-byte aligned (written)
  *   other arguments as in kvq_rot_quant_fwd.
  */
-kvq_status kvq_decode_step(const uint16_t *x_new, uint8_t *packed,
-                           float *scales, int64_t n_heads, int64_t cap,
-                           int64_t pos, int32_t d, int32_t group,
-                           const int8_t *signs, kvq_rot rot, uint16_t *out,
-                           kvq_stream stream);
+KVQ_API kvq_status kvq_decode_step(const uint16_t *x_new, uint8_t *packed,
+                                   float *scales, int64_t n_heads, int64_t cap,
+                                   int64_t pos, int32_t d, int32_t group,
+                                   const int8_t *signs, kvq_rot rot, uint16_t *out,
+                                   kvq_stream stream);
 
 /*
  * Decode step with a dequantized-prefix cache and an fp16 tail ("Quantization
@@ -224,12 +233,12 @@ kvq_status kvq_decode_step(const uint16_t *x_new, uint8_t *packed,
  *   window  1 <= window <= 4096 (16 in the pages' design)
  *   other arguments as in kvq_rot_quant_fwd.
  */
-kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *packed,
-                                    float *scales, uint16_t *kv,
-                                    int64_t n_heads, int64_t cap, int64_t pos,
-                                    int32_t window, int32_t d, int32_t group,
-                                    const int8_t *signs, kvq_rot rot,
-                                    kvq_stream stream);
+KVQ_API kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *packed,
+                                            float *scales, uint16_t *kv,
+                                            int64_t n_heads, int64_t cap, int64_t pos,
+                                            int32_t window, int32_t d, int32_t group,
+                                            const int8_t *signs, kvq_rot rot,
+                                            kvq_stream stream);
 
 /*
  * Decode attention that reads the int4 cache directly ("Day 9 -
@@ -257,15 +266,15 @@ kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *packed,
  *   signs, rot, d, group as in kvq_rot_quant_fwd (the D and R the cache
  *   was written with).
  */
-kvq_status kvq_attend_decode(const uint16_t *q, const uint8_t *k_packed,
-                             const float *k_scales, const uint8_t *v_packed,
-                             const float *v_scales, int64_t n_kv_heads,
-                             int32_t n_q, int64_t cap, int64_t len, int32_t d,
-                             int32_t group, const int8_t *signs, kvq_rot rot,
-                             float sm_scale, uint16_t *out, kvq_stream stream);
+KVQ_API kvq_status kvq_attend_decode(const uint16_t *q, const uint8_t *k_packed,
+                                     const float *k_scales, const uint8_t *v_packed,
+                                     const float *v_scales, int64_t n_kv_heads,
+                                     int32_t n_q, int64_t cap, int64_t len, int32_t d,
+                                     int32_t group, const int8_t *signs, kvq_rot rot,
+                                     float sm_scale, uint16_t *out, kvq_stream stream);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
-const char *kvq_status_string(kvq_status s);
+KVQ_API const char *kvq_status_string(kvq_status s);
 
 /*
  * Device-side error word of the current device.  The kernels bound every
@@ -274,10 +283,10 @@ const char *kvq_status_string(kvq_status s);
  * synchronizes the device, returns KVQ_OK or the recorded status, and clears
  * the word when `clear` is non-zero.
  */
-kvq_status kvq_device_status(int32_t clear);
+KVQ_API kvq_status kvq_device_status(int32_t clear);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
-int32_t kvq_version(void);
+KVQ_API int32_t kvq_version(void);
 
 #ifdef __cplusplus
 }

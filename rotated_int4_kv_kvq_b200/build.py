@@ -25,8 +25,13 @@ LIB = os.path.join(PKG, "libkvq.so")
 
 SOURCES = ["kvq_api.cu", "kvq_d64.cu", "kvq_d128.cu", "kvq_d256.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# Hidden visibility: only the C API (KVQ_API in include/kvq.h) is exported.
+# Otherwise the function-local statics of inline and template code are
+# exported as process-wide unique symbols and shared by every build of the
+# library loaded into one process.
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
-         "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+         "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr", "-I", INCLUDE,
+         "-I", CSRC]
 # Extra nvcc flags (e.g. -D tuning overrides) and an alternative output
 # path, for building variants side by side.
 EXTRA = os.environ.get("KVQ_NVCC_EXTRA", "").split()

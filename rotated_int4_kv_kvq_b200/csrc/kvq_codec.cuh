@@ -40,12 +40,12 @@ namespace kvq {
 // Round the SRFT join outputs with packed f32x2 multiply-adds (1) or one
 // scalar multiply-add per value (0).
 #ifndef KVQ_SRFT_QFMA2
-#define KVQ_SRFT_QFMA2 0
+#define KVQ_SRFT_QFMA2 1
 #endif
 // Flip and widen the fp16 inputs with one mixed-precision multiply-add per
 // sample (1), or XOR the sign bits and widen (0).
 #ifndef KVQ_MIXED_CVT
-#define KVQ_MIXED_CVT 0
+#define KVQ_MIXED_CVT 1
 #endif
 
 constexpr int kWarps = 4;

@@ -203,3 +203,18 @@ def test_calls_run_on_the_tensors_device(kvq):
         kvq.kvq_rot_quant_fwd(x1, s0, kvq.SRFT, g)
     with pytest.raises(ValueError, match="stream"):
         kvq.kvq_rot_quant_fwd(x1, s1, kvq.SRFT, g, stream=torch.cuda.Stream(device=0))
+
+
+def test_library_exports_only_the_declared_functions(kvq):
+    """Built with hidden visibility: the dynamic symbol table holds the C API
+    and nothing else (no inline or template statics that a second build of
+    the library in the same process would share)."""
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    r = subprocess.run([nm, "-D", "--defined-only", kvq.LIB_PATH], capture_output=True,
+                       text=True, check=True)
+    names = {line.split()[-1] for line in r.stdout.splitlines() if line.strip()}
+    assert names == set(declared_functions())
