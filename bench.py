@@ -520,7 +520,7 @@ def cpu_legs(kvq, S, dev, peak_unused=None):
     codes for each."""
     import oracle.kvq_oracle as O
     per_step_bytes, total_s, flips = 0, 0.0, {}
-    rows_per_d = {64: 16384, 128: 16384, 256: 8192}
+    rows_per_d = {64: 262144, 128: 262144, 256: 131072}  # about 10 s on 16 cores
     for d, T in S.items():
         idx = torch.from_numpy(W.sample_rows(T.n, rows_per_d[d], seed=7 + d)).to(dev)
         xg = T.x[idx].contiguous()

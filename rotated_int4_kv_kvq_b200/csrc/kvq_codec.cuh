@@ -42,6 +42,11 @@ namespace kvq {
 #ifndef KVQ_SRFT_QFMA2
 #define KVQ_SRFT_QFMA2 1
 #endif
+// Warp barriers between batches of 8 lambda factor loads in the inverse (1)
+// or none (0).
+#ifndef KVQ_LAM_FENCE
+#define KVQ_LAM_FENCE 1
+#endif
 // Flip and widen the fp16 inputs with one mixed-precision multiply-add per
 // sample (1), or XOR the sign bits and widen (0).
 #ifndef KVQ_MIXED_CVT
@@ -242,13 +247,17 @@ __device__ __forceinline__ void load_x(uint32_t tile, int row, int t, uint32_t m
   }
 }
 
-template <class C>
+// Thread t's words of the output row into the swizzled tile, XOR-ed with
+// the store-side sign masks (MASK), or as they are (the lambda path has
+// applied the signs in fp32 already).
+template <class C, bool MASK = true>
 __device__ __forceinline__ void store_x(uint32_t tile, int row, int t, uint32_t mask,
                                         const uint32_t (&xw)[C::NW]) {
 #pragma unroll
   for (int c = 0; c < C::NW / 4; ++c) {
     const int gc = t * (C::NW / 4) + c;
-    const uint4 m = lds128(mask + c * 16);
+    uint4 m = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (MASK) m = lds128(mask + c * 16);
     sts128(tile + (gc / 8) * C::SLAB + sw128(row, gc % 8), xw[4 * c] ^ m.x,
            xw[4 * c + 1] ^ m.y, xw[4 * c + 2] ^ m.z, xw[4 * c + 3] ^ m.w);
   }
@@ -543,8 +552,9 @@ __device__ __forceinline__ void pair_join_inv(const f2 (&Y)[C::P], int t, f2 (&Z
 // inverse of rotate_fwd's unnormalized map up to the factor 1/KAPPA^2) yields
 // u itself.  Words of a two-lane codelet output that carry polarity -1 are
 // corrected by the store-side sign mask.
-// With LAM, the values are multiplied by the store-side 1/lambda pairs at
-// `lam` (shared memory) before the fp16 rounding.
+// With LAM, the values are multiplied by the store-side factor pairs at
+// `lam` (shared memory: sign / lambda, see fill_lambda) before the fp16
+// rounding, and the store path applies no sign mask.
 template <class C, bool LAM = false>
 __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[C::NW],
                                            uint32_t lam = 0) {
@@ -556,7 +566,7 @@ __device__ __forceinline__ void rotate_inv(f2 (&Y)[C::P], int t, uint32_t (&xw)[
   // loads are not moved across it, so at most 8 lambda pairs are live at a
   // time (loaded all at once, they pushed the register demand into spills).
   auto fence = [&](int j) {
-    if constexpr (LAM) {
+    if constexpr (LAM && KVQ_LAM_FENCE) {
       if (j % 8 == 7) __syncwarp();
     }
   };
@@ -819,17 +829,42 @@ __device__ __forceinline__ void lambda_channels(int t, int j, bool store, int& c
   }
 }
 
-// s_lam[0, d/2): lambda pairs of the load side, s_lam[d/2, d): 1/lambda
-// pairs of the store side, NW pairs per thread role t.
+// Store-side factor of lane l (0: low, 1: high sample) of pair p that thread
+// role tp converts to fp16 in rotate_inv: the sign the store mask would
+// apply to that sample (D and the inverse codelet's output polarity) over
+// lambda of its channel.  Thread-pair SRFT: pairs p < NW/2 stay with the
+// thread and land in words 2p + l of its half of the row (low half for
+// thread 0, high half for thread 1); pairs p >= NW/2 go to the partner as
+// its words 2(p - NW/2) + l (high half for thread 0, low half for thread 1).
 template <class C>
-__device__ __forceinline__ void fill_lambda(const float* lambda, f2* s_lam) {
+__device__ __forceinline__ float store_factor(const int8_t* signs, const float* lambda, int tp,
+                                              int p, int l) {
+  int t = tp, w = p, h = l;
+  if constexpr (C::PAIR_RFFT) {
+    const bool own = p < C::NW / 2;
+    t = own ? tp : 1 - tp;
+    w = 2 * (own ? p : p - C::NW / 2) + l;
+    h = own ? (t == 0 ? 0 : 1) : (t == 0 ? 1 : 0);
+  }
+  const uint32_t m = store_mask_word<C>(signs, t, w);
+  const bool neg = (m >> (h ? 31 : 15)) & 1u;
+  const float inv = 1.0f / lambda[2 * (t * C::NW + w) + h];
+  return neg ? -inv : inv;
+}
+
+// s_lam[0, d/2): lambda pairs of the load side, s_lam[d/2, d): the
+// store-side factor pairs (sign / lambda, see store_factor), NW pairs per
+// thread role t.  With lambda the store path applies the signs through these
+// factors in fp32 and skips the fp16 sign-bit XOR.
+template <class C>
+__device__ __forceinline__ void fill_lambda(const int8_t* signs, const float* lambda, f2* s_lam) {
   for (int i = threadIdx.x; i < C::D / 2; i += blockDim.x) {
     const int t = i / C::NW, j = i % C::NW;
     int c0, c1;
     lambda_channels<C>(t, j, false, c0, c1);
     s_lam[i] = mk2(lambda[c0], lambda[c1]);
-    lambda_channels<C>(t, j, true, c0, c1);
-    s_lam[C::D / 2 + i] = mk2(1.0f / lambda[c0], 1.0f / lambda[c1]);
+    s_lam[C::D / 2 + i] = mk2(store_factor<C>(signs, lambda, t, j, 0),
+                              store_factor<C>(signs, lambda, t, j, 1));
   }
 }
 
@@ -927,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t bars = smem_u32(&bars_sm[warp][0]);
 
   fill_sign_masks<C>(a.signs, s_mask);
-  if constexpr (LAM) fill_lambda<C>(a.lambda, s_lam);
+  if constexpr (LAM) fill_lambda<C>(a.signs, a.lambda, s_lam);
   if (lane == 0) {
     for (int s = 0; s < S_IN; ++s) mbar_init(bars + 8u * s, 1);
     fence_mbar_init();
@@ -1029,7 +1064,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t bars = smem_u32(&bars_sm[warp][0]);
 
   fill_sign_masks<C>(a.signs, s_mask);
-  if constexpr (LAM) fill_lambda<C>(a.lambda, s_lam);
+  if constexpr (LAM) fill_lambda<C>(a.signs, a.lambda, s_lam);
   if (lane == 0) {
     for (int s = 0; s < S_IN; ++s) mbar_init(bars + 8u * s, 1);
     fence_mbar_init();
@@ -1091,7 +1126,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (lane == 0) bulk_wait_read<S_OUT - 1>();
     __syncwarp();
     const uint32_t xdst = xbuf + uint32_t(o * C::XTILE);
-    store_x<C>(xdst, row, t, mask_st, xw);
+    store_x<C, !LAM>(xdst, row, t, mask_st, xw);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {

@@ -44,6 +44,9 @@ struct InvLaunch {
 #define KVQ_WIDE_MAX_ROWS (int64_t(1) << 16)
 #endif
 constexpr int64_t kWideMaxRows = KVQ_WIDE_MAX_ROWS;
+// The one-warp-per-vector kernel maps rows with 32-bit reciprocal
+// multiplies that are exact for at most 2^16 rows per call.
+static_assert(kWideMaxRows <= (int64_t(1) << 16), "wide decode calls are limited to 2^16 rows");
 
 struct DecodeWideLaunch {
   const uint16_t* x_new;

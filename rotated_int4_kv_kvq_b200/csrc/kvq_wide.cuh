@@ -445,11 +445,19 @@ __global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const Dec
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int64_t total = a.n_heads * (a.pos + 1);
-  // item -> (head, row): the new token of every head first, then cached rows
+  // item -> (head, row): the new token of every head first, then cached rows.
+  // This kernel runs calls of at most 2^16 rows, so the cached-row index n
+  // and pos fit 16 bits and n / pos = umulhi(n, ceil(2^32 / pos)) exactly
+  // (checked for every pos in [2, 2^16] and n < 2^16), a multiply instead of
+  // a 64-bit division per row.
+  const uint32_t P = uint32_t(a.pos);
+  const uint32_t recip = P > 1u ? 0xFFFFFFFFu / P + 1u : 0u;
   auto where = [&](int64_t it, int64_t& head, int64_t& row) {
     const bool fresh = it < a.n_heads;
-    head = fresh ? it : (it - a.n_heads) / a.pos;
-    row = fresh ? a.pos : (it - a.n_heads) % a.pos;
+    const uint32_t n = uint32_t(it - a.n_heads);
+    const uint32_t q = P > 1u ? __umulhi(n, recip) : n;
+    head = fresh ? it : int64_t(q);
+    row = fresh ? a.pos : int64_t(n - q * P);
     return fresh;
   };
   // the codes and scale of a cached row are loaded one item ahead, so their
