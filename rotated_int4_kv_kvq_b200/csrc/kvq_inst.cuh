@@ -282,7 +282,8 @@ cudaError_t decode_wide_one(const DecodeWideLaunch& L) {
   int occ;
   cudaError_t e = wide_occupancy<kern>(&occ);
   if (e != cudaSuccess) return e;
-  DecodeWideArgs a{L.x_new, L.packed, L.scales, L.out, L.signs, L.n_heads, L.cap, L.pos};
+  DecodeWideArgs a{L.x_new, L.packed, L.scales, L.out, L.signs, L.n_heads, L.cap, L.pos,
+                   wide_pos_recip(L.pos)};
   return launch_pdl(kern, wide_grid(L.n_heads * (L.pos + 1), L.sm_count, occ), kWideThreads, 0,
                     L.stream, a);
 }

@@ -286,7 +286,15 @@ struct DecodeWideArgs {
   uint16_t* out;          // [n_heads][pos+1][d]
   const int8_t* signs;
   int64_t n_heads, cap, pos;
+  uint32_t pos_recip;     // ceil(2^32 / pos) for pos >= 2 (wide_pos_recip)
 };
+
+// The multiplier that divides a cached-row index n < 2^16 by pos exactly:
+// n / pos = umulhi(n, ceil(2^32 / pos)) for 2 <= pos <= 2^16 (checked for
+// every such pos and n).  Computed once per call on the host.
+inline uint32_t wide_pos_recip(int64_t pos) {
+  return pos > 1 ? uint32_t(0xFFFFFFFFull / uint64_t(pos)) + 1u : 0u;
+}
 
 // Loads through the read-only path unless RO is false (rows this kernel
 // also writes).
@@ -447,15 +455,13 @@ __global__ void __launch_bounds__(kWideThreads) kvq_decode_wide_kernel(const Dec
   const int64_t total = a.n_heads * (a.pos + 1);
   // item -> (head, row): the new token of every head first, then cached rows.
   // This kernel runs calls of at most 2^16 rows, so the cached-row index n
-  // and pos fit 16 bits and n / pos = umulhi(n, ceil(2^32 / pos)) exactly
-  // (checked for every pos in [2, 2^16] and n < 2^16), a multiply instead of
-  // a 64-bit division per row.
+  // and pos fit 16 bits and n / pos is one multiply by the host's
+  // reciprocal (wide_pos_recip) instead of a 64-bit division per row.
   const uint32_t P = uint32_t(a.pos);
-  const uint32_t recip = P > 1u ? 0xFFFFFFFFu / P + 1u : 0u;
   auto where = [&](int64_t it, int64_t& head, int64_t& row) {
     const bool fresh = it < a.n_heads;
     const uint32_t n = uint32_t(it - a.n_heads);
-    const uint32_t q = P > 1u ? __umulhi(n, recip) : n;
+    const uint32_t q = P > 1u ? __umulhi(n, a.pos_recip) : n;
     head = fresh ? it : int64_t(q);
     row = fresh ? a.pos : int64_t(n - q * P);
     return fresh;
