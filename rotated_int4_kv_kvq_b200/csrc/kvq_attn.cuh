@@ -127,6 +127,114 @@ __device__ __forceinline__ void attn_unpack(uint32_t code, f2 (&c)[C]) {
   for (int j = 0; j < C; ++j) c[j] = sub2(q[j], magic);
 }
 
+// Merges the per-warp partials in shared memory (slot w of s_part: m and l
+// of every query, then the NQ x D accumulated rotated coordinates, written
+// before the call) across the block and the cluster: the block's triple goes
+// to its slot 0, the cluster's blocks merge into slot 1 of block 0, a slice
+// each, and block 0 rotates every query's result back and stores it.
+template <int D, int ROT, int NQ>
+__device__ __forceinline__ void attn_merge_store(const AttnArgs& a, float* s_part,
+                                                 cooperative_groups::cluster_group& cluster,
+                                                 int rank, int nblk, int64_t head, int warp,
+                                                 int lane, const WideLane<D, ROT>& L) {
+  using P = Wide<D, ROT>;
+  constexpr int W = P::W, C = P::C;
+  using AP = AttnPartial<D, NQ>;
+  const int k2 = L.k2;
+  float* stage = s_part + kAttnWarps * AP::FLOATS;
+  __syncthreads();
+  // per query, the weight f_w = 2^(m_w - max_w m_w) of every warp's partial,
+  // formed once (warp qi for query qi, lane w for warp w's partial, max and
+  // sum by shuffles); then thread i merges element i of every (query,
+  // coordinate) and leaves the block's triple in warp slot 0
+  __shared__ float s_bw[kAttnWarps * NQ];
+  static_assert(NQ <= kAttnWarps && kAttnWarps <= 32, "one warp per query, a lane per warp");
+  if (warp < NQ) {
+    const int qi = warp;
+    const bool has = lane < kAttnWarps;
+    const float mw = has ? s_part[lane * AP::FLOATS + 2 * qi] : -INFINITY;
+    const float lw = has ? s_part[lane * AP::FLOATS + 2 * qi + 1] : 0.0f;
+    float mm = mw;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
+    const float f = mw == -INFINITY ? 0.0f : exp2f(mw - mm);
+    float ls = f * lw;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+    if (has) s_bw[lane * NQ + qi] = f;
+    if (lane == 0) {  // m, l of every slot are still being read: stage them
+      stage[2 * qi] = mm;
+      stage[2 * qi + 1] = ls;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
+    const int qi = e / D;
+    float accv = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w)
+      accv += s_bw[w * NQ + qi] * s_part[w * AP::FLOATS + 2 * NQ + e];
+    s_part[2 * NQ + e] = accv;  // slot 0 (warp 0's region): read only by this thread
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * NQ) s_part[threadIdx.x] = stage[threadIdx.x];
+  cluster.sync();  // every block's triple is in its slot 0
+
+  // ---- the cluster's blocks merge into slot 1 of block 0, a slice each ----
+  // weights of every block's triple per query: f_b / sum_b f_b l_b with
+  // f_b = 2^(m_b - max_b m_b); each block reads the (m, l) pairs once, one
+  // remote read per thread, and forms the weights in its own shared memory
+  __shared__ float s_w[kAttnMaxCluster * NQ];
+  __shared__ float s_l[kAttnMaxCluster * NQ];
+  for (int i = threadIdx.x; i < nblk * NQ; i += kAttnThreads) {
+    const float* src = cluster.map_shared_rank(s_part, i / NQ);
+    s_w[i] = src[2 * (i % NQ)];
+    s_l[i] = src[2 * (i % NQ) + 1];
+  }
+  __syncthreads();
+  static_assert(kAttnMaxCluster <= 32, "a lane per block of the cluster");
+  if (warp < NQ) {  // warp qi: lane b forms block b's weight, max and sum by shuffles
+    const int qi = warp;
+    const bool has = lane < nblk;
+    const float mb = has ? s_w[lane * NQ + qi] : -INFINITY;
+    const float lb = has ? s_l[lane * NQ + qi] : 0.0f;
+    float mm = mb;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
+    const float f = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
+    float ls = f * lb;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+    if (has) s_w[lane * NQ + qi] = f * (1.0f / ls);
+  }
+  __syncthreads();
+  {
+    float* fin = cluster.map_shared_rank(s_part, 0) + AP::FLOATS;
+    constexpr int NE = NQ * D;
+    const int per = (NE + nblk - 1) / nblk;
+    const int e_end = (rank + 1) * per < NE ? (rank + 1) * per : NE;
+    for (int e = rank * per + threadIdx.x; e < e_end; e += kAttnThreads) {
+      const int qi = e / D;
+      float accv = 0.0f;
+#pragma unroll 4
+      for (int b = 0; b < nblk; ++b)
+        accv += s_w[b * NQ + qi] * cluster.map_shared_rank(s_part, b)[2 * NQ + e];
+      fin[2 * NQ + e] = accv;
+    }
+  }
+  cluster.sync();  // block 0's slot 1 is complete; remote reads done, others may exit
+  if (rank == 0 && warp < a.nq) {
+    const int qi = warp;
+    const float* fin = s_part + AP::FLOATS + 2 * NQ + qi * D;
+    float Y[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) Y[w] = fin[k2 * W + w] * P::KAPPA;
+    uint32_t xo[C];
+    wide_rotate_inv<D, ROT>(Y, L, xo);
+    wide_store_words<D, ROT>(a.out + (head * a.nq + qi) * D, L, xo);
+  }
+}
+
 template <int D, int ROT, int NQ>
 __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArgs a) {
   namespace cg = cooperative_groups;
@@ -323,8 +431,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
   pdl_release();
   __syncthreads();  // the staging rings become the merge area
 
-  // ---- merge the warps of this block ----
-  float* stage = s_part + kAttnWarps * AP::FLOATS;
+  // ---- this warp's partial into its merge slot ----
   float* mine = s_part + warp * AP::FLOATS;
   if (lane % TB == 0) {
     mine[2 * (lane / TB)] = m;
@@ -338,97 +445,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
       dst[0] = lo2(acc[qi][j]);
       dst[1] = hi2(acc[qi][j]);
     }
-  __syncthreads();
-  // per query, the weight f_w = 2^(m_w - max_w m_w) of every warp's partial,
-  // formed once (warp qi for query qi, lane w for warp w's partial, max and
-  // sum by shuffles); then thread i merges element i of every (query,
-  // coordinate) and leaves the block's triple in warp slot 0
-  __shared__ float s_bw[kAttnWarps * NQ];
-  static_assert(NQ <= kAttnWarps && kAttnWarps <= 32, "one warp per query, a lane per warp");
-  if (warp < NQ) {
-    const int qi = warp;
-    const bool has = lane < kAttnWarps;
-    const float mw = has ? s_part[lane * AP::FLOATS + 2 * qi] : -INFINITY;
-    const float lw = has ? s_part[lane * AP::FLOATS + 2 * qi + 1] : 0.0f;
-    float mm = mw;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
-    const float f = mw == -INFINITY ? 0.0f : exp2f(mw - mm);
-    float ls = f * lw;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
-    if (has) s_bw[lane * NQ + qi] = f;
-    if (lane == 0) {  // m, l of every slot are still being read: stage them
-      stage[2 * qi] = mm;
-      stage[2 * qi + 1] = ls;
-    }
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < NQ * D; e += kAttnThreads) {
-    const int qi = e / D;
-    float accv = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w)
-      accv += s_bw[w * NQ + qi] * s_part[w * AP::FLOATS + 2 * NQ + e];
-    s_part[2 * NQ + e] = accv;  // slot 0 (warp 0's region): read only by this thread
-  }
-  __syncthreads();
-  if (threadIdx.x < 2 * NQ) s_part[threadIdx.x] = stage[threadIdx.x];
-  cluster.sync();  // every block's triple is in its slot 0
-
-  // ---- the cluster's blocks merge into slot 1 of block 0, a slice each ----
-  // weights of every block's triple per query: f_b / sum_b f_b l_b with
-  // f_b = 2^(m_b - max_b m_b); each block reads the (m, l) pairs once, one
-  // remote read per thread, and forms the weights in its own shared memory
-  __shared__ float s_w[kAttnMaxCluster * NQ];
-  __shared__ float s_l[kAttnMaxCluster * NQ];
-  for (int i = threadIdx.x; i < nblk * NQ; i += kAttnThreads) {
-    const float* src = cluster.map_shared_rank(s_part, i / NQ);
-    s_w[i] = src[2 * (i % NQ)];
-    s_l[i] = src[2 * (i % NQ) + 1];
-  }
-  __syncthreads();
-  static_assert(kAttnMaxCluster <= 32, "a lane per block of the cluster");
-  if (warp < NQ) {  // warp qi: lane b forms block b's weight, max and sum by shuffles
-    const int qi = warp;
-    const bool has = lane < nblk;
-    const float mb = has ? s_w[lane * NQ + qi] : -INFINITY;
-    const float lb = has ? s_l[lane * NQ + qi] : 0.0f;
-    float mm = mb;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
-    const float f = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
-    float ls = f * lb;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
-    if (has) s_w[lane * NQ + qi] = f * (1.0f / ls);
-  }
-  __syncthreads();
-  {
-    float* fin = cluster.map_shared_rank(s_part, 0) + AP::FLOATS;
-    constexpr int NE = NQ * D;
-    const int per = (NE + nblk - 1) / nblk;
-    const int e_end = (rank + 1) * per < NE ? (rank + 1) * per : NE;
-    for (int e = rank * per + threadIdx.x; e < e_end; e += kAttnThreads) {
-      const int qi = e / D;
-      float accv = 0.0f;
-#pragma unroll 4
-      for (int b = 0; b < nblk; ++b)
-        accv += s_w[b * NQ + qi] * cluster.map_shared_rank(s_part, b)[2 * NQ + e];
-      fin[2 * NQ + e] = accv;
-    }
-  }
-  cluster.sync();  // block 0's slot 1 is complete; remote reads done, others may exit
-  if (rank == 0 && warp < a.nq) {
-    const int qi = warp;
-    const float* fin = s_part + AP::FLOATS + 2 * NQ + qi * D;
-    float Y[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) Y[w] = fin[k2 * W + w] * P::KAPPA;
-    uint32_t xo[C];
-    wide_rotate_inv<D, ROT>(Y, L, xo);
-    wide_store_words<D, ROT>(a.out + (head * a.nq + qi) * D, L, xo);
-  }
+  attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
 // Dynamic shared memory of kvq_attn_kernel.

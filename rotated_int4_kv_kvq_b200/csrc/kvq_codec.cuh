@@ -11,7 +11,10 @@
 //    with conflict-free 128-bit shared loads.
 //  * Each thread holds its vector (or half of it) in registers and runs the
 //    whole step there: sign flip, rotation (FFT / FWHT, plus one exchange
-//    stage through warp shuffles when TPV = 2), absmax, round, pack.
+//    stage through warp shuffles when TPV = 2), absmax, round, pack.  The
+//    forward flips and widens each fp16 input with one mixed-precision
+//    multiply-add by an fp16 +-1 (the inverse XORs the fp16 sign bits of its
+//    output words, or folds the signs into its lambda factors).
 //  * SRFT: an fp16 word is an (even, odd) sample pair, so one generated
 //    two-lane real-FFT codelet in packed fp32x2 transforms both parity halves
 //    at once (half the issue slots of a scalar codelet) and a radix-2 join
