@@ -1040,13 +1040,17 @@ def graph_time_us(fn, reps=20):
 
 def run_attention_suite(kvq, dev, peak):
     """Decode attention reading the int4 cache: the Gemma-3-1B step (26
-    layers, 1 KV head with 4 queries, d = g = 256) as a graph of 26 calls, and
-    one SmolLM2-1.7B-shaped layer (32 KV heads, 1 query each, d = g = 64) for
-    throughput against the HBM roofline (codes + scales of K and V)."""
+    layers, 1 KV head with 4 queries, d = g = 256) as a graph of 26 calls, one
+    SmolLM2-1.7B-shaped layer (32 KV heads, 1 query each, d = g = 64), and the
+    same layers batched over several sequences in one call (the KV heads of
+    all sequences as the call's heads), for throughput against the HBM
+    roofline (codes + scales of K and V)."""
     out = []
     gen = torch.Generator(device=dev).manual_seed(21)
     cases = [("gemma-3-1b step", 26, 1, 4, 256, 256, (256, 1024, 2048, 4096)),
-             ("smollm2-1.7b layer", 1, 32, 1, 64, 64, (1024, 4096, 16384))]
+             ("smollm2-1.7b layer", 1, 32, 1, 64, 64, (1024, 4096, 16384)),
+             ("gemma-3-1b layer x 64 sequences", 1, 64, 4, 256, 256, (4096,)),
+             ("smollm2-1.7b layer x 16 sequences", 1, 512, 1, 64, 64, (16384,))]
     for name, layers, heads, nq, d, g, lens in cases:
         cap = max(lens)
         signs = torch.from_numpy(W.make_signs(d)).to(dev)
@@ -1058,6 +1062,7 @@ def run_attention_suite(kvq, dev, peak):
                     x = (torch.randn((heads * cap, d), generator=gen, device=dev)).half()
                     p, s = kvq.kvq_rot_quant_fwd(x, signs, rot, g)
                     c += [p.reshape(heads, cap, -1), s.reshape(heads, cap, -1)]
+                    del x
                 q = torch.randn((heads, nq, d), generator=gen, device=dev).half()
                 o = torch.empty((heads, nq, d), dtype=torch.float16, device=dev)
                 caches.append((q, c, o))
@@ -1068,7 +1073,7 @@ def run_attention_suite(kvq, dev, peak):
                 us = graph_time_us(fn)
                 byts = layers * heads * n * 2 * fwd_bytes(d, g) - layers * heads * n * 2 * 2 * d
                 out.append({"workload": name, "rot": "srft" if rot == 0 else "srht",
-                            "len": n, "graph_us": us, "calls": layers,
+                            "len": n, "kv_heads": heads, "graph_us": us, "calls": layers,
                             "algo_bytes": byts, "algo_gbs": byts / (us * 1e-6) / 1e9,
                             "frac": byts / (us * 1e-6) / 1e9 / peak})
             del caches

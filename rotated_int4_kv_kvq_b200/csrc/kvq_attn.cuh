@@ -36,6 +36,17 @@ constexpr int kAttnChunk = 32;   // tokens per staged chunk of a warp
 constexpr int kAttnStages = 2;   // chunks in flight per warp
 constexpr int kAttnMaxCluster = 16;  // blocks per KV head at most
 
+// Iterations of a warp's tokens in flight in the lane-pair kernel (cp.async
+// into shared memory; 0: plain loads into registers, two tokens ahead).
+#ifndef KVQ_ATTN_PAIR_STAGES
+#define KVQ_ATTN_PAIR_STAGES 3
+#endif
+// Unpack codes in the lane-pair kernel through fp16 and mixed-precision
+// multiply-adds (1) or byte permutes into offset floats (0).
+#ifndef KVQ_ATTN_MIXED_UNPACK
+#define KVQ_ATTN_MIXED_UNPACK 1
+#endif
+
 // Asynchronous global -> shared copies (cp.async); `bytes` < size zero-fills
 // the rest and 0 reads nothing.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int bytes) {
@@ -445,6 +456,260 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
       dst[0] = lo2(acc[qi][j]);
       dst[1] = hi2(acc[qi][j]);
     }
+  attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
+}
+
+// Dynamic shared memory of kvq_attn_pair_kernel: the merge slots (which also
+// hold the rotated query before the token loop), then the warps' stages.
+template <int D>
+constexpr int attn_pair_merge_bytes() {
+  constexpr int merge = (kAttnWarps * AttnPartial<D, 1>::FLOATS + 2) * 4;
+  return ((merge > D * 4 ? merge : D * 4) + 15) / 16 * 16;
+}
+template <int D>
+constexpr int attn_pair_smem_bytes() {
+  return attn_pair_merge_bytes<D>() +
+         kAttnWarps * KVQ_ATTN_PAIR_STAGES * (2 * 32 * (D / 2) + 32 * 16);
+}
+
+// Decode attention at d = 64 with one query per KV head (multi-head caches
+// such as SmolLM2's): a pair of lanes per token instead of a warp.  Lane h
+// of a pair holds rotated coordinates [32h, 32h + 32) of the query; for each
+// of its tokens it reads that half's 16 code bytes and scale of K and of V
+// with one 128-bit and one 32-bit load each (consecutive pairs read
+// consecutive rows), forms its partial dot product, and the pair adds the two
+// halves with one shuffle.  A pair takes two tokens per iteration, 128 rows
+// apart, with all eight loads issued before either is used.  Each lane keeps
+// its own online softmax (base 2, one update per two tokens) and
+// accumulator.  After the loop the 16 pairs of a warp merge by shuffles
+// (a reduce-scatter leaves each lane two coordinates), and the block and the
+// cluster merge as in kvq_attn_kernel.  Per token a warp issues about a
+// third of the instructions of the warp-per-token layout, whose lanes hold
+// only two coordinates each at d = 64.
+template <int D, int ROT>
+__global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const AttnArgs a) {
+  static_assert(D == 64, "a lane pair per token: 32 coordinates per lane");
+  namespace cg = cooperative_groups;
+  constexpr int NQ = 1;
+  using P = Wide<D, ROT>;
+  constexpr int W = P::W, C = P::C;
+  constexpr int HC = D / 2;   // coordinates per lane
+  constexpr int NP = HC / 2;  // f2 pairs per lane
+  constexpr int QB = HC / 2;  // code bytes per lane and token
+  [[maybe_unused]] constexpr int kPairs = kAttnThreads / 2;
+  using AP = AttnPartial<D, NQ>;
+  extern __shared__ __align__(16) float s_part[];
+
+  pdl_wait();  // no global access before the previous kernel completes
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = int(cluster.block_rank());
+  const int nblk = int(cluster.num_blocks());
+  const int64_t head = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WideLane<D, ROT> L;
+  L.init(a.signs, lane);
+  const int h = lane & 1;
+  const int ng = D / a.group;      // scales per token (1 or 2)
+  const int sh = ng == 2 ? h : 0;  // the scale of this lane's half
+
+  // this block's tokens
+  const int64_t per = (a.len + nblk - 1) / nblk;
+  const int64_t t_begin = int64_t(rank) * per;
+  const int64_t t_end = t_begin + per < a.len ? t_begin + per : a.len;
+  const uint32_t n_tok = uint32_t(t_end > t_begin ? t_end - t_begin : 0);
+  const uint32_t pmask = 3u << (lane & 30);
+#if KVQ_ATTN_PAIR_STAGES > 0
+  // Iteration i of warp w covers tokens ob + [0, 32) of the block's range,
+  // ob = 256 i + 32 w; pair pp = lane / 2 takes ob + pp and ob + 16 + pp.
+  // Each lane copies its own halves of the two tokens' K and V codes and
+  // their scales into a stage of its warp (cp.async, KVQ_ATTN_PAIR_STAGES
+  // stages) and reads back only what it copied, so completion is per lane.
+  constexpr int S = KVQ_ATTN_PAIR_STAGES;
+  constexpr int CB = 32 * (D / 2);         // code bytes of 32 tokens (K or V)
+  constexpr int STAGE = 2 * CB + 32 * 16;  // then (sk0, sv0, sk1, sv1) per lane
+  const int64_t row0 = head * a.cap + t_begin;
+  const uint8_t* kb = a.k_packed + row0 * (D / 2) + QB * h;
+  const uint8_t* vb = a.v_packed + row0 * (D / 2) + QB * h;
+  const float* ks = a.k_scales + row0 * ng + sh;
+  const float* vs = a.v_scales + row0 * ng + sh;
+  const int pp = lane >> 1;
+  const uint32_t stages =
+      smem_u32(s_part) + uint32_t(attn_pair_merge_bytes<D>() + warp * S * STAGE);
+  auto issue = [&](uint32_t ob, int s) {
+    if (ob < n_tok) {
+      const uint32_t st = stages + uint32_t(s * STAGE);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t o = ob + 16u * j + uint32_t(pp);
+        const uint32_t r = o < n_tok ? o : ob;  // out of range: zero fill from a valid row
+        const int n16 = o < n_tok ? 16 : 0, n4 = o < n_tok ? 4 : 0;
+        cp_async16(st + uint32_t(16 * (32 * j + lane)), kb + size_t(r) * (D / 2), n16);
+        cp_async16(st + uint32_t(CB + 16 * (32 * j + lane)), vb + size_t(r) * (D / 2), n16);
+        cp_async4(st + uint32_t(2 * CB + 16 * lane + 8 * j), ks + size_t(r) * ng, n4);
+        cp_async4(st + uint32_t(2 * CB + 16 * lane + 8 * j + 4), vs + size_t(r) * ng, n4);
+      }
+    }
+    cp_async_commit();  // one group per iteration, empty past the range
+  };
+#pragma unroll
+  for (int s = 0; s < S - 1; ++s) issue(uint32_t(32 * warp + 256 * s), s);
+#else
+  const uint8_t* kb = a.k_packed + head * a.cap * (D / 2) + QB * h;
+  const uint8_t* vb = a.v_packed + head * a.cap * (D / 2) + QB * h;
+  const float* ks = a.k_scales + head * a.cap * ng + sh;
+  const float* vs = a.v_scales + head * a.cap * ng + sh;
+#endif
+
+  // the rotated, pre-scaled query: warp 0 rotates it into shared memory,
+  // every lane takes its half
+  if (warp == 0) {
+    uint32_t xw[C];
+    wide_load_words<D, ROT>(a.q + head * D, L, xw);
+    float Y[W];
+    wide_rotate_fwd<D, ROT>(xw, L, Y);
+#pragma unroll
+    for (int w = 0; w < W; ++w) s_part[L.k2 * W + w] = Y[w] * a.qscale;
+  }
+  __syncthreads();
+  f2 qr[NP];
+#pragma unroll
+  for (int j = 0; j < NP; ++j) qr[j] = mk2(s_part[HC * h + 2 * j], s_part[HC * h + 2 * j + 1]);
+  __syncthreads();  // the query slots become merge slots
+
+  [[maybe_unused]] const f2 magic = mk2(kUnpackMagic, kUnpackMagic);
+  float m = -INFINITY, l = 0.0f;
+  f2 acc[NP];
+#pragma unroll
+  for (int j = 0; j < NP; ++j) acc[j] = mk2(0.0f, 0.0f);
+  // half of the K dot product of one token (times its scale)
+  auto kdot = [&](const uint4& kc, float sk) {
+    const uint32_t kw[4] = {kc.x, kc.y, kc.z, kc.w};
+    f2 d2 = mk2(0.0f, 0.0f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      f2 c[4];
+#if KVQ_ATTN_MIXED_UNPACK
+      unpack8_signed(kw[w], c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d2 = fma2(qr[4 * w + i], c[i], d2);
+#else
+      unpack8(kw[w], c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d2 = fma2(qr[4 * w + i], sub2(c[i], magic), d2);
+#endif
+    }
+    return (lo2(d2) + hi2(d2)) * sk;
+  };
+  auto vacc = [&](const uint4& vc, float wv) {
+    const uint32_t vw[4] = {vc.x, vc.y, vc.z, vc.w};
+    const f2 w2 = mk2(wv, wv);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      f2 c[4];
+#if KVQ_ATTN_MIXED_UNPACK
+      unpack8_signed(vw[w], c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[4 * w + i] = fma2(w2, c[i], acc[4 * w + i]);
+#else
+      unpack8(vw[w], c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[4 * w + i] = fma2(w2, sub2(c[i], magic), acc[4 * w + i]);
+#endif
+    }
+  };
+  // one online-softmax update for two scored tokens (s1 = -inf: no second)
+  auto update = [&](float s0, float s1, const uint4& vc0, float sv0, const uint4& vc1, float sv1) {
+    const float mx = fmaxf(s0, s1);
+    if (mx > m) {  // a new maximum: rescale what has accumulated (m = -inf: zeros)
+      const float corr = exp2f(m - mx);
+      const f2 c2 = mk2(corr, corr);
+      l *= corr;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) acc[j] = mul2(acc[j], c2);
+      m = mx;
+    }
+    const float p0 = exp2f(s0 - m), p1 = exp2f(s1 - m);
+    l += p0 + p1;
+    vacc(vc0, p0 * sv0);
+    vacc(vc1, p1 * sv1);
+  };
+#if KVQ_ATTN_PAIR_STAGES > 0
+  int s_use = 0;
+  for (uint32_t ob = uint32_t(32 * warp); ob < n_tok; ob += 256u) {
+    issue(ob + 256u * (S - 1), s_use == 0 ? S - 1 : s_use - 1);
+    cp_async_wait<S - 1>();  // this lane's copies of this iteration have landed
+    const uint32_t st = stages + uint32_t(s_use * STAGE);
+    s_use = s_use == S - 1 ? 0 : s_use + 1;
+    if (ob + pp < n_tok) {  // a pair with no token left skips the work
+      const bool two = ob + 16u + pp < n_tok;
+      const uint4 kc0 = lds128(st + uint32_t(16 * lane));
+      const uint4 kc1 = lds128(st + uint32_t(16 * (32 + lane)));
+      const uint4 sc = lds128(st + uint32_t(2 * CB + 16 * lane));
+      const uint4 vc0 = lds128(st + uint32_t(CB + 16 * lane));
+      const uint4 vc1 = lds128(st + uint32_t(CB + 16 * (32 + lane)));
+      const float part0 = kdot(kc0, __uint_as_float(sc.x));
+      const float part1 = kdot(kc1, __uint_as_float(sc.z));
+      const float s0 = part0 + __shfl_xor_sync(pmask, part0, 1);
+      const float s1r = part1 + __shfl_xor_sync(pmask, part1, 1);
+      update(s0, two ? s1r : -INFINITY, vc0, __uint_as_float(sc.y), vc1, __uint_as_float(sc.w));
+    }
+  }
+  cp_async_wait<0>();
+#else
+  // two tokens per pair and iteration, t and t + kPairs: their eight loads
+  // are issued together (a token past the block's range reads row t again
+  // and gets weight 0)
+  for (uint32_t o = uint32_t(threadIdx.x >> 1); o < n_tok; o += 2 * kPairs) {
+    const uint32_t t0 = uint32_t(t_begin) + o;
+    const bool two = o + kPairs < n_tok;
+    const uint32_t t1 = two ? t0 + kPairs : t0;
+    const uint4 kc0 = __ldg(reinterpret_cast<const uint4*>(kb + size_t(t0) * (D / 2)));
+    const uint4 kc1 = __ldg(reinterpret_cast<const uint4*>(kb + size_t(t1) * (D / 2)));
+    const float sk0 = __ldg(ks + size_t(t0) * ng), sk1 = __ldg(ks + size_t(t1) * ng);
+    const uint4 vc0 = __ldg(reinterpret_cast<const uint4*>(vb + size_t(t0) * (D / 2)));
+    const uint4 vc1 = __ldg(reinterpret_cast<const uint4*>(vb + size_t(t1) * (D / 2)));
+    const float sv0 = __ldg(vs + size_t(t0) * ng), sv1 = __ldg(vs + size_t(t1) * ng);
+    const float part0 = kdot(kc0, sk0), part1 = kdot(kc1, sk1);
+    const float s0 = part0 + __shfl_xor_sync(pmask, part0, 1);
+    const float s1r = part1 + __shfl_xor_sync(pmask, part1, 1);
+    update(s0, two ? s1r : -INFINITY, vc0, sv0, vc1, sv1);
+  }
+#endif
+  pdl_release();
+
+  // ---- the warp's 16 pairs into one partial ----
+  float mm = m;
+#pragma unroll
+  for (int o = 2; o <= 16; o <<= 1) mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
+  const float f = m == -INFINITY ? 0.0f : exp2f(m - mm);
+  float ls = l * f;
+#pragma unroll
+  for (int o = 2; o <= 16; o <<= 1) ls += __shfl_xor_sync(kFull, ls, o);
+  float v[HC];
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    v[2 * j] = lo2(acc[j]) * f;
+    v[2 * j + 1] = hi2(acc[j]) * f;
+  }
+  // reduce-scatter over lane bits 4..1 (the pair index): 32 -> 2 values,
+  // lane keeps coordinates HC h + (lane & 30) + {0, 1}
+#pragma unroll
+  for (int o = 16, n = HC / 2; o >= 2; o >>= 1, n >>= 1) {
+    const bool upper = lane & o;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float send = upper ? v[j] : v[j + n];
+      const float keep = upper ? v[j + n] : v[j];
+      v[j] = keep + __shfl_xor_sync(kFull, send, o);
+    }
+  }
+  float* mine = s_part + warp * AP::FLOATS;
+  mine[2 * NQ + HC * h + (lane & 30)] = v[0];
+  mine[2 * NQ + HC * h + (lane & 30) + 1] = v[1];
+  if (lane == 0) {
+    mine[0] = mm;
+    mine[1] = ls;
+  }
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 

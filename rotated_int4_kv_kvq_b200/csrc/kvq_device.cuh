@@ -438,6 +438,42 @@ __device__ __forceinline__ void unpack8(uint32_t w, f2 (&q)[4]) {
                __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + j)));
 }
 
+// Codes of a packed word as 4 pairs of exact signed floats (pair j = codes
+// 2j, 2j+1).  One logic op puts two nibbles into an fp16 pair (1032 + q for
+// a low nibble, 1152 + 16 q for a high one), and one mixed-precision
+// multiply-add per code (f16 x f16 + f32 -> f32, exact) removes the offset:
+// five integer and eight floating-point instructions per word, where
+// unpack8 and a packed subtraction take eleven integer and four.
+__device__ __forceinline__ void unpack8_signed(uint32_t w, f2 (&q)[4]) {
+  const uint32_t w8 = w >> 8;
+  const uint32_t l0 = (w & 0x000F000Fu) ^ 0x64086408u;   // codes 0, 4
+  const uint32_t h0 = (w & 0x00F000F0u) ^ 0x64806480u;   // codes 1, 5
+  const uint32_t l1 = (w8 & 0x000F000Fu) ^ 0x64086408u;  // codes 2, 6
+  const uint32_t h1 = (w8 & 0x00F000F0u) ^ 0x64806480u;  // codes 3, 7
+  float c0, c1, c2, c3, c4, c5, c6, c7;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1, d0, d1, e0, e1, one, s16;\n\t"
+      "mov.b16 one, 0x3C00;\n\t"
+      "mov.b16 s16, 0x2C00;\n\t"
+      "mov.b32 {a0, a1}, %8;\n\t"
+      "mov.b32 {b0, b1}, %9;\n\t"
+      "mov.b32 {d0, d1}, %10;\n\t"
+      "mov.b32 {e0, e1}, %11;\n\t"
+      "fma.rn.f32.f16 %0, a0, one, 0fC4810000;\n\t"
+      "fma.rn.f32.f16 %1, b0, s16, 0fC2900000;\n\t"
+      "fma.rn.f32.f16 %2, d0, one, 0fC4810000;\n\t"
+      "fma.rn.f32.f16 %3, e0, s16, 0fC2900000;\n\t"
+      "fma.rn.f32.f16 %4, a1, one, 0fC4810000;\n\t"
+      "fma.rn.f32.f16 %5, b1, s16, 0fC2900000;\n\t"
+      "fma.rn.f32.f16 %6, d1, one, 0fC4810000;\n\t"
+      "fma.rn.f32.f16 %7, e1, s16, 0fC2900000;\n\t}"
+      : "=f"(c0), "=f"(c1), "=f"(c2), "=f"(c3), "=f"(c4), "=f"(c5), "=f"(c6), "=f"(c7)
+      : "r"(l0), "r"(h0), "r"(l1), "r"(h1));
+  q[0] = mk2(c0, c1);
+  q[1] = mk2(c2, c3);
+  q[2] = mk2(c4, c5);
+  q[3] = mk2(c6, c7);
+}
+
 // 32 codes (the low BITS bits of each magic-rounded float, two's
 // complement) as BITS words of a little-endian bitstream: code i occupies
 // bits [BITS i, BITS i + BITS).

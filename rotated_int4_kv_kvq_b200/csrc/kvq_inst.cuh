@@ -45,6 +45,9 @@ static __device__ unsigned g_status;
 #ifndef KVQ_ATTN_MAX_CLUSTER
 #define KVQ_ATTN_MAX_CLUSTER 16
 #endif
+#ifndef KVQ_ATTN_PAIR_TOKENS
+#define KVQ_ATTN_PAIR_TOKENS 8
+#endif
 #ifndef KVQ_ATTN_ROWS_PER_WARP
 #define KVQ_ATTN_ROWS_PER_WARP 4
 #endif
@@ -300,48 +303,44 @@ cudaError_t window_one(const WindowLaunch& L) {
   return launch_pdl(kern, wide_grid(rows, L.sm_count, occ), kWideThreads, 0, L.stream, a);
 }
 
-template <int D, int ROT, int NQ>
-cudaError_t attn_nq(int group, const AttnLaunch& L) {
-  constexpr auto kern = kvq_attn_kernel<D, ROT, NQ>;
-  constexpr int smem = attn_smem_bytes<D, NQ>();
-  int max_cluster;
-  {
-    static int maxc[kMaxDevices];
-    static std::mutex mu;
-    int dev;
-    cudaError_t e = current_device(&dev);
+// Largest cluster (blocks per KV head) the attention kernel `Kern` may use on
+// the current device: up to 16 where the device can co-schedule them, else 8
+// (looked up once per kernel and device; also opts the kernel into its
+// dynamic shared memory).
+template <auto Kern>
+cudaError_t attn_max_cluster(int smem, int* out) {
+  static int maxc[kMaxDevices];
+  static std::mutex mu;
+  int dev;
+  cudaError_t e = current_device(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  if (maxc[dev] == 0) {
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    std::lock_guard<std::mutex> g(mu);
-    if (maxc[dev] == 0) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      // clusters of up to 16 blocks where the device can co-schedule them
-      static_assert(KVQ_ATTN_MAX_CLUSTER <= kAttnMaxCluster, "attention merge weights");
-      int c = std::min(8, KVQ_ATTN_MAX_CLUSTER);
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-          cudaSuccess) {
-        cudaLaunchConfig_t q = {};
-        q.gridDim = dim3(16, 1, 1);
-        q.blockDim = dim3(kAttnThreads, 1, 1);
-        q.dynamicSmemBytes = smem;
-        int best = 0;
-        if (cudaOccupancyMaxPotentialClusterSize(&best, kern, &q) == cudaSuccess && best >= 8)
-          c = std::min(std::min(best, 16), KVQ_ATTN_MAX_CLUSTER);
-      }
-      cudaGetLastError();
-      maxc[dev] = c;
+    static_assert(KVQ_ATTN_MAX_CLUSTER <= kAttnMaxCluster, "attention merge weights");
+    int c = std::min(8, KVQ_ATTN_MAX_CLUSTER);
+    if (cudaFuncSetAttribute(Kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(16, 1, 1);
+      q.blockDim = dim3(kAttnThreads, 1, 1);
+      q.dynamicSmemBytes = smem;
+      int best = 0;
+      if (cudaOccupancyMaxPotentialClusterSize(&best, Kern, &q) == cudaSuccess && best >= 8)
+        c = std::min(std::min(best, 16), KVQ_ATTN_MAX_CLUSTER);
     }
-    max_cluster = maxc[dev];
+    cudaGetLastError();
+    maxc[dev] = c;
   }
-  // blocks per KV head (one cluster): about KVQ_ATTN_ROWS_PER_WARP rows per
-  // warp, and no more than the SMs left per head (one resident block per SM)
-  constexpr int64_t per_block = int64_t(kAttnWarps) * KVQ_ATTN_ROWS_PER_WARP;
-  const int64_t by_len = (L.len + per_block - 1) / per_block;
-  const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
-  const int cl = int(std::max<int64_t>(
-      1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
-  AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
-             L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
+  *out = maxc[dev];
+  return cudaSuccess;
+}
+
+// One cluster of `cl` blocks per KV head.
+template <typename... KArgs>
+cudaError_t attn_launch(void (*kern)(KArgs...), int cl, int smem, const AttnLaunch& L,
+                        const AttnArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(cl), unsigned(L.n_kv), 1);
   cfg.blockDim = dim3(kAttnThreads, 1, 1);
@@ -359,8 +358,49 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
+// d = 64 with one query per KV head: the lane-pair kernel, about
+// KVQ_ATTN_PAIR_TOKENS tokens per pair and block, up to two blocks per SM.
+template <int D, int ROT>
+cudaError_t attn_pair(int group, const AttnLaunch& L) {
+  constexpr auto kern = kvq_attn_pair_kernel<D, ROT>;
+  constexpr int smem = attn_pair_smem_bytes<D>();
+  int max_cluster;
+  cudaError_t e = attn_max_cluster<kern>(smem, &max_cluster);
+  if (e != cudaSuccess) return e;
+  constexpr int64_t per_block = int64_t(kAttnThreads / 2) * KVQ_ATTN_PAIR_TOKENS;
+  const int64_t by_len = (L.len + per_block - 1) / per_block;
+  const int64_t by_sms = std::max<int64_t>(1, 2 * int64_t(L.sm_count) / std::max<int64_t>(1, L.n_kv));
+  const int cl = int(std::max<int64_t>(
+      1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
+             L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
+  return attn_launch(kern, cl, smem, L, a);
+}
+
+template <int D, int ROT, int NQ>
+cudaError_t attn_nq(int group, const AttnLaunch& L) {
+  constexpr auto kern = kvq_attn_kernel<D, ROT, NQ>;
+  constexpr int smem = attn_smem_bytes<D, NQ>();
+  int max_cluster;
+  cudaError_t e = attn_max_cluster<kern>(smem, &max_cluster);
+  if (e != cudaSuccess) return e;
+  // blocks per KV head (one cluster): about KVQ_ATTN_ROWS_PER_WARP rows per
+  // warp, and no more than the SMs left per head (one resident block per SM)
+  constexpr int64_t per_block = int64_t(kAttnWarps) * KVQ_ATTN_ROWS_PER_WARP;
+  const int64_t by_len = (L.len + per_block - 1) / per_block;
+  const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
+  const int cl = int(std::max<int64_t>(
+      1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
+             L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
+  return attn_launch(kern, cl, smem, L, a);
+}
+
 template <int D, int ROT>
 cudaError_t attn_rot(int group, const AttnLaunch& L) {
+  if constexpr (D == 64) {
+    if (L.nq == 1) return attn_pair<D, ROT>(group, L);
+  }
   if (L.nq <= 1) return attn_nq<D, ROT, 1>(group, L);
   if (L.nq <= 2) return attn_nq<D, ROT, 2>(group, L);
   if (L.nq <= 4) return attn_nq<D, ROT, 4>(group, L);

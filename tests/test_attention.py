@@ -83,3 +83,16 @@ def test_attention_gemma_shape(kvq):
 def test_attention_many_heads(kvq):
     """SmolLM2-1.7B-like layer: 32 KV heads, one query each, d = g = 64."""
     run_case(kvq, 64, 64, O.SRFT, heads=32, nq=1, length=1024, seed=10)
+
+
+@pytest.mark.parametrize("group", [32, 64])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("heads,length,scale", [(1, 4096, None), (3, 9001, None), (2, 2048, 0.0),
+                                                (5, 1500, 3.0), (40, 777, None), (1, 1, None),
+                                                (300, 2500, None)])
+def test_attention_lane_pair_d64(kvq, group, rot, heads, length, scale):
+    """d = 64 with one query per KV head (the lane-pair kernel): single blocks
+    and clusters of several blocks, ragged token splits, flat and sharp
+    softmax, a single row, and more heads than SMs (one block per head)."""
+    run_case(kvq, 64, group, rot, heads=heads, nq=1, length=length, sm_scale=scale,
+             seed=heads + length + group)
