@@ -66,13 +66,14 @@ def run_eager_and_graph(chain, init, tensors):
     del graph
 
 
-@pytest.mark.parametrize("d,group", [(64, 64), (256, 256), (128, 32)])
+@pytest.mark.parametrize("d,group,nq", [(64, 64, 4), (64, 64, 1), (256, 256, 4), (128, 32, 4)])
 @pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
-def test_consecutive_decode_steps_and_attention(kvq, d, group, rot):
+def test_consecutive_decode_steps_and_attention(kvq, d, group, nq, rot):
     """Each position: decode step on the K heads, on the V heads (each
     appends row pos and decodes rows [0, pos]), then attention over
-    pos + 1 rows that include the two rows just written."""
-    heads, cap, pre, steps, nq = 2, 48, 20, 12, 4
+    pos + 1 rows that include the two rows just written (d = 64 with one
+    query per head runs the lane-pair attention kernel)."""
+    heads, cap, pre, steps = 2, 48, 20, 12
     signs = torch.from_numpy(W.make_signs(d)).cuda()
     k_hist, k0p, k0s = state(d, group, heads, cap, pre, 11 + d, kvq, rot, signs)
     v_hist, v0p, v0s = state(d, group, heads, cap, pre, 12 + d, kvq, rot, signs)
