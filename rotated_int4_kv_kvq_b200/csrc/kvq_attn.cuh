@@ -536,8 +536,21 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   const uint32_t stages =
       smem_u32(s_part) + uint32_t(attn_pair_merge_bytes<D>() + warp * S * STAGE);
   auto issue = [&](uint32_t ob, int s) {
-    if (ob < n_tok) {
-      const uint32_t st = stages + uint32_t(s * STAGE);
+    const uint32_t st = stages + uint32_t(s * STAGE);
+    if (ob + 32u <= n_tok) {  // the warp's 32 tokens all in range: no clamps
+      const size_t r = size_t(ob) + uint32_t(pp);
+      const uint8_t* kp = kb + r * (D / 2);
+      const uint8_t* vp = vb + r * (D / 2);
+      const float* ksp = ks + r * ng;
+      const float* vsp = vs + r * ng;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        cp_async16(st + uint32_t(16 * (32 * j + lane)), kp + 16 * j * (D / 2), 16);
+        cp_async16(st + uint32_t(CB + 16 * (32 * j + lane)), vp + 16 * j * (D / 2), 16);
+        cp_async4(st + uint32_t(2 * CB + 16 * lane + 8 * j), ksp + 16 * j * ng, 4);
+        cp_async4(st + uint32_t(2 * CB + 16 * lane + 8 * j + 4), vsp + 16 * j * ng, 4);
+      }
+    } else if (ob < n_tok) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const uint32_t o = ob + 16u * j + uint32_t(pp);
