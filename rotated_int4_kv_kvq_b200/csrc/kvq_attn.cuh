@@ -726,6 +726,302 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
+// ------------------------- tensor-core decode attention (d = g = 256, 4 queries) ---
+//
+// The Gemma-3-1B shape: 4 queries per KV head, d = g = 256.  Per warp and
+// chunk of 16 tokens the rotated-domain scores and the accumulation run on
+// the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//   scores           S = K Q^T:  M = 16 tokens, N = 8 = 4 queries x (hi, lo),
+//                                K = 256 rotated coordinates (16 steps);
+//   accumulation     O^T = V^T P'^T:  M = 256 coordinates (16 tiles), N = the
+//                                same 8 columns, K = the 16 tokens.
+// int4 codes are exact in bf16; each query (and each weight p s_V) is split
+// into a bf16 high part and a bf16 remainder, the two columns of its pair, so
+// products are exact and the two column sums, added at the end, carry ~16
+// significant bits (error ~2^-17 relative, well under the fp16 output's).
+// With one scale per token (g = d) a token's K scale multiplies its score
+// after the dot product and its V scale folds into its weight.
+//
+// Fragments (PTX ISA, m16n8k16 with 16-bit inputs; lane = 4 g + c): A holds
+// rows g and g + 8, columns 2c, 2c + 1 and 2c + 8, 2c + 9; B rows (the K
+// index) 2c, 2c + 1, 2c + 8, 2c + 9 of column g; C rows g, g + 8, columns 2c,
+// 2c + 1.  The coordinates of a step may be any permutation applied to both
+// operands: thread c's K operand comes from bytes [32c, 32c + 32) of a code
+// row, a 32-bit word giving two steps (see attn_tc_kword); a V tile mt takes
+// row g from the low nibble and row g + 8 from the high nibble of byte
+// 16 g + mt.  Column n = 2q + h: query q, part h (0 high, 1 remainder), so
+// thread (g, c) holds the score of query c for tokens g and g + 8 and
+// accumulates query c.
+
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// (lo, hi) -> bf16x2 with lo in the low half, rounded to nearest.
+__device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// The codes of the low nibbles of bytes 0 and 2 of x as an exact bf16 pair:
+// (x & 0x000F000F) ^ 0x43084308 is 128 + (n ^ 8) = 136 + q, minus 136.
+__device__ __forceinline__ uint32_t attn_tc_lo(uint32_t x) {
+  return bf16x2_fma((x & 0x000F000Fu) ^ 0x43084308u, 0x3F803F80u, 0xC308C308u);
+}
+// ... of the high nibbles of bytes 0 and 2 (shifted down first: bf16 has
+// only 7 mantissa bits, so a nibble at bits 4-7 would reach the exponent).
+__device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x) { return attn_tc_lo(x >> 4); }
+
+// Physical coordinate of K-index slot `e` (0: 2c, 1: 2c + 1, 2: 2c + 8,
+// 3: 2c + 9) of step s for thread c: word s / 2 of the thread's 32 bytes
+// holds coordinates 2b .. 2b + 7 (b = 32 c + 4 (s / 2)); even steps take the
+// nibbles of bytes b and b + 2, odd steps those of b + 1 and b + 3.
+__device__ __forceinline__ int attn_tc_coord(int c, int s, int e) {
+  const int b = 32 * c + 4 * (s >> 1);
+  const int base = 2 * b + 2 * (s & 1) + (e >> 1);  // low (e < 2) or high nibble
+  return base + 4 * (e & 1);                        // byte b (+1) or b + 2 (+3)
+}
+
+constexpr int kTcChunk = 16;   // tokens per warp and chunk
+constexpr int kTcStages = 3;   // chunks in flight per warp
+constexpr int kTcRow = 128;    // code bytes per row (d = 256)
+// staged chunk: K rows | V rows (16 x 128 B, 16-byte chunks swizzled by the
+// token index) | K scales | V scales
+constexpr int kTcStage = 2 * kTcChunk * kTcRow + 2 * kTcChunk * 4;
+
+template <int ROT>
+__global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const AttnArgs a) {
+  namespace cg = cooperative_groups;
+  constexpr int D = 256, NQ = 4;
+  using P = Wide<D, ROT>;
+  constexpr int W = P::W;
+  using AP = AttnPartial<D, NQ>;
+  extern __shared__ __align__(16) float s_part[];  // staging, queries; then merge slots
+
+  pdl_wait();  // no global access before the previous kernel completes
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = int(cluster.block_rank());
+  const int nblk = int(cluster.num_blocks());
+  const int64_t head = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  WideLane<D, ROT> L;
+  L.init(a.signs, lane);
+
+  // this block's tokens, then this warp's contiguous share (whole chunks)
+  const int64_t per = (a.len + nblk - 1) / nblk;
+  const int64_t t_begin = int64_t(rank) * per;
+  const int64_t t_end = t_begin + per < a.len ? t_begin + per : a.len;
+  const int64_t per_w =
+      ((t_end - t_begin + kAttnWarps - 1) / kAttnWarps + kTcChunk - 1) / kTcChunk * kTcChunk;
+  const int64_t w_begin = t_begin + int64_t(warp) * per_w;
+  const int64_t w_end = w_begin + per_w < t_end ? w_begin + per_w : t_end;
+  const int n_w = int(w_end > w_begin ? w_end - w_begin : 0);
+  const int nchunk = (n_w + kTcChunk - 1) / kTcChunk;
+  const uint8_t* kbase = a.k_packed + head * a.cap * kTcRow;
+  const uint8_t* vbase = a.v_packed + head * a.cap * kTcRow;
+  const float* ksc = a.k_scales + head * a.cap;
+  const float* vsc = a.v_scales + head * a.cap;
+
+  const uint32_t ring = smem_u32(s_part) + uint32_t(warp * kTcStages * kTcStage);
+  auto issue = [&](int ci) {
+    if (ci < nchunk) {
+      const uint32_t st = ring + uint32_t((ci % kTcStages) * kTcStage);
+      const int64_t r0 = w_begin + int64_t(ci) * kTcChunk;
+      const int rows = n_w - ci * kTcChunk < kTcChunk ? n_w - ci * kTcChunk : kTcChunk;
+#pragma unroll
+      for (int i = lane; i < kTcChunk * (kTcRow / 16); i += 32) {  // 4 pieces per lane
+        const int t = i >> 3, ch = i & 7;
+        const bool ok = t < rows;
+        const int64_t off = ok ? (r0 + t) * kTcRow + ch * 16 : r0 * kTcRow;
+        const uint32_t dst = uint32_t(t * kTcRow + ((ch ^ (t & 7)) << 4));
+        cp_async16(st + dst, kbase + off, ok ? 16 : 0);
+        cp_async16(st + uint32_t(kTcChunk * kTcRow) + dst, vbase + off, ok ? 16 : 0);
+      }
+      {
+        const int t = lane & 15;
+        const bool ok = t < rows;
+        const float* src = (lane < 16 ? ksc : vsc) + (ok ? r0 + t : r0);
+        cp_async4(st + uint32_t(2 * kTcChunk * kTcRow + lane * 4), src, ok ? 4 : 0);
+      }
+    }
+    cp_async_commit();  // possibly empty: keeps the group count uniform
+  };
+#pragma unroll
+  for (int ci = 0; ci < kTcStages - 1; ++ci) issue(ci);
+
+  // rotated, pre-scaled queries (score = <qr, y_K> in log2 units): warp w
+  // rotates query w into shared memory after the staging rings
+  float* s_q = s_part + kAttnWarps * kTcStages * (kTcStage / 4);
+  float* s_p = s_q + NQ * D;  // per warp: weights [4 queries][16 tokens]
+  if (warp < NQ) {
+    uint32_t xw[P::C];
+    if (warp < a.nq) {
+      wide_load_words<D, ROT>(a.q + (head * a.nq + warp) * D, L, xw);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P::C; ++j) xw[j] = 0u;
+    }
+    float Y[W];
+    wide_rotate_fwd<D, ROT>(xw, L, Y);
+#pragma unroll
+    for (int w = 0; w < W; ++w) s_q[warp * D + L.k2 * W + w] = Y[w] * a.qscale;
+  }
+  __syncthreads();
+  // B operand of the scores: column g = 2 q + h of step s, rows (slots)
+  // 2c, 2c + 1 (qb[s][0]) and 2c + 8, 2c + 9 (qb[s][1])
+  uint32_t qb[16][2];
+  {
+    const float* qrow = s_q + (g >> 1) * D;
+    const bool rem = g & 1;
+#pragma unroll
+    for (int s = 0; s < 16; ++s)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float v0 = qrow[attn_tc_coord(c, s, 2 * r)];
+        const float v1 = qrow[attn_tc_coord(c, s, 2 * r + 1)];
+        const uint32_t hi = bf16x2_pack(v0, v1);
+        const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+        qb[s][r] = rem ? bf16x2_pack(v0 - h0, v1 - h1) : hi;
+      }
+  }
+
+  float m = -INFINITY, l = 0.0f;  // of query c
+  float o[16][4];                 // O^T tiles: coordinates 2 (16 g + mt) (+1), columns 2c, 2c + 1
+#pragma unroll
+  for (int mt = 0; mt < 16; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[mt][i] = 0.0f;
+  const uint32_t pw = smem_u32(s_p) + uint32_t(warp * NQ * kTcChunk * 4);
+
+  for (int ci = 0; ci < nchunk; ++ci) {
+    cp_async_wait<kTcStages - 2>();
+    __syncwarp();  // the chunk's copies (by every lane) are visible
+    const uint32_t st = ring + uint32_t((ci % kTcStages) * kTcStage);
+    const uint32_t kst = st, vst = st + uint32_t(kTcChunk * kTcRow);
+    const uint32_t sst = st + uint32_t(2 * kTcChunk * kTcRow);
+    const int rows = n_w - ci * kTcChunk < kTcChunk ? n_w - ci * kTcChunk : kTcChunk;
+
+    // ---- scores: tokens g and g + 8, query c ----
+    float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {  // bytes [32c + 16hh, +16) of tokens g and g + 8
+      const uint4 k0 = lds128(kst + uint32_t(g * kTcRow + (((2 * c + hh) ^ (g & 7)) << 4)));
+      const uint4 k8 = lds128(kst + uint32_t((g + 8) * kTcRow + (((2 * c + hh) ^ (g & 7)) << 4)));
+      const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
+      const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w};
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+        const int s = 2 * (4 * hh + wi);
+        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi]), attn_tc_lo(w8[wi]), attn_tc_hi(w0[wi]),
+                          attn_tc_hi(w8[wi]), qb[s][0], qb[s][1]);
+        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi] >> 8), attn_tc_lo(w8[wi] >> 8),
+                          attn_tc_hi(w0[wi] >> 8), attn_tc_hi(w8[wi] >> 8), qb[s + 1][0],
+                          qb[s + 1][1]);
+      }
+    }
+    const float sk0 = __uint_as_float(lds32(sst + uint32_t(g * 4)));
+    const float sk8 = __uint_as_float(lds32(sst + uint32_t((g + 8) * 4)));
+    const float sc0 = g < rows ? (sacc[0] + sacc[1]) * sk0 : -INFINITY;
+    const float sc8 = g + 8 < rows ? (sacc[2] + sacc[3]) * sk8 : -INFINITY;
+
+    // ---- online softmax of query c over the chunk (lanes c, c + 4, ...) ----
+    float mx = fmaxf(sc0, sc8);
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, msk));
+    const float m_new = fmaxf(m, mx);  // finite: the chunk holds a valid token
+    const float corr = exp2f(m - m_new);
+    const float p0 = exp2f(sc0 - m_new), p8 = exp2f(sc8 - m_new);
+    float ps = p0 + p8;
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) ps += __shfl_xor_sync(kFull, ps, msk);
+    l = l * corr + ps;
+    m = m_new;
+    if (__any_sync(kFull, corr != 1.0f)) {
+#pragma unroll
+      for (int mt = 0; mt < 16; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[mt][i] *= corr;
+    }
+    // weights p s_V by (query, token) through shared memory, then the B
+    // operand: column g = 2 q + h, tokens 2c, 2c + 1 and 2c + 8, 2c + 9
+    const float sv0 = __uint_as_float(lds32(sst + uint32_t((kTcChunk + g) * 4)));
+    const float sv8 = __uint_as_float(lds32(sst + uint32_t((kTcChunk + g + 8) * 4)));
+    sts32(pw + uint32_t((c * kTcChunk + g) * 4), __float_as_uint(p0 * sv0));
+    sts32(pw + uint32_t((c * kTcChunk + g + 8) * 4), __float_as_uint(p8 * sv8));
+    __syncwarp();
+    uint32_t pb[2];
+    {
+      const bool rem = g & 1;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint2 v = lds64(pw + uint32_t(((g >> 1) * kTcChunk + 2 * c + 8 * r) * 4));
+        const float v0 = __uint_as_float(v.x), v1 = __uint_as_float(v.y);
+        const uint32_t hi = bf16x2_pack(v0, v1);
+        const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+        pb[r] = rem ? bf16x2_pack(v0 - h0, v1 - h1) : hi;
+      }
+    }
+
+    // ---- accumulation: V rows 2c, 2c + 1, 2c + 8, 2c + 9, bytes [16g, 16g + 16) ----
+    {
+      auto vrow = [&](int t) { return lds128(vst + uint32_t(t * kTcRow + ((g ^ (t & 7)) << 4))); };
+      const uint4 va = vrow(2 * c), vb = vrow(2 * c + 1);
+      const uint4 vc = vrow(2 * c + 8), vd = vrow(2 * c + 9);
+      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+      const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+#pragma unroll
+      for (int mt = 0; mt < 16; ++mt) {
+        const uint32_t sel = uint32_t(mt & 3) | (uint32_t(4 + (mt & 3)) << 8);
+        const uint32_t x01 = __byte_perm(wa[mt >> 2], wb[mt >> 2], sel);  // tokens 2c, 2c + 1
+        const uint32_t x89 = __byte_perm(wc[mt >> 2], wd[mt >> 2], sel);  // 2c + 8, 2c + 9
+        mma_bf16_m16n8k16(o[mt], attn_tc_lo(x01), attn_tc_hi(x01), attn_tc_lo(x89),
+                          attn_tc_hi(x89), pb[0], pb[1]);
+      }
+    }
+    __syncwarp();  // the stage and the weights are consumed before they are refilled
+    issue(ci + kTcStages - 1);
+  }
+  cp_async_wait<0>();
+  pdl_release();
+  __syncthreads();  // the staging rings become the merge area
+
+  // ---- this warp's partial into its merge slot (y order) ----
+  float* mine = s_part + warp * AP::FLOATS;
+  if (g == 0) {
+    mine[2 * c] = m;
+    mine[2 * c + 1] = l;
+  }
+#pragma unroll
+  for (int mt = 0; mt < 16; ++mt) {
+    const int y = 2 * (16 * g + mt);
+    mine[2 * NQ + c * D + y] = o[mt][0] + o[mt][1];
+    mine[2 * NQ + c * D + y + 1] = o[mt][2] + o[mt][3];
+  }
+  attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
+}
+
+// Dynamic shared memory of kvq_attn_tc_kernel.
+constexpr int attn_tc_smem_bytes() {
+  constexpr int merge = (kAttnWarps * AttnPartial<256, 4>::FLOATS + 2 * 4) * 4;
+  constexpr int staging =
+      kAttnWarps * kTcStages * kTcStage + 4 * 256 * 4 + kAttnWarps * 4 * kTcChunk * 4;
+  return merge > staging ? merge : staging;
+}
+
 // Dynamic shared memory of kvq_attn_kernel.
 template <int D, int NQ>
 constexpr int attn_smem_bytes() {

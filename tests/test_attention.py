@@ -96,3 +96,15 @@ def test_attention_lane_pair_d64(kvq, group, rot, heads, length, scale):
     softmax, a single row, and more heads than SMs (one block per head)."""
     run_case(kvq, 64, group, rot, heads=heads, nq=1, length=length, sm_scale=scale,
              seed=heads + length + group)
+
+
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("heads,nq,length,scale", [(1, 4, 1, None), (2, 3, 15, None), (1, 4, 16, None),
+                                                   (3, 4, 17, 2.0), (1, 3, 4096, None), (2, 4, 5003, 0.0),
+                                                   (64, 4, 700, None), (1, 4, 33, 6.0)])
+def test_attention_tensor_core_d256(kvq, rot, heads, nq, length, scale):
+    """d = g = 256 with 3 or 4 queries per KV head (the tensor-core kernel):
+    single tokens, partial and whole 16-token chunks, several blocks per
+    head, flat and sharp softmax, more heads than one block each."""
+    run_case(kvq, 256, 256, rot, heads=heads, nq=nq, length=length, sm_scale=scale,
+             seed=heads * 7 + nq + length)
