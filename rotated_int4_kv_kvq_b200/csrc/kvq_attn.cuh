@@ -726,15 +726,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
-// ------------------------- tensor-core decode attention (d = g = 256, 4 queries) ---
+// ----------------------------- tensor-core decode attention (g = d, up to 4 queries) ---
 //
-// The Gemma-3-1B shape: 4 queries per KV head, d = g = 256.  Per warp and
-// chunk of 16 tokens the rotated-domain scores and the accumulation run on
-// the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+// One scale per token (g = d), up to 4 queries per KV head (e.g. the
+// Gemma-3-1B shape, d = 256 with 4 queries).  Per warp and chunk of 16
+// tokens the rotated-domain scores and the accumulation run on the tensor
+// cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
 //   scores           S = K Q^T:  M = 16 tokens, N = 8 = 4 queries x (hi, lo),
-//                                K = 256 rotated coordinates (16 steps);
-//   accumulation     O^T = V^T P'^T:  M = 256 coordinates (16 tiles), N = the
-//                                same 8 columns, K = the 16 tokens.
+//                                K = d rotated coordinates (d / 16 steps);
+//   accumulation     O^T = V^T P'^T:  M = d coordinates (d / 16 tiles), N =
+//                                the same 8 columns, K = the 16 tokens.
 // int4 codes are exact in bf16; each query (and each weight p s_V) is split
 // into a bf16 high part and a bf16 remainder, the two columns of its pair, so
 // products are exact and the two column sums, added at the end, carry ~16
@@ -746,10 +747,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
 // rows g and g + 8, columns 2c, 2c + 1 and 2c + 8, 2c + 9; B rows (the K
 // index) 2c, 2c + 1, 2c + 8, 2c + 9 of column g; C rows g, g + 8, columns 2c,
 // 2c + 1.  The coordinates of a step may be any permutation applied to both
-// operands: thread c's K operand comes from bytes [32c, 32c + 32) of a code
-// row, a 32-bit word giving two steps (see attn_tc_kword); a V tile mt takes
-// row g from the low nibble and row g + 8 from the high nibble of byte
-// 16 g + mt.  Column n = 2q + h: query q, part h (0 high, 1 remainder), so
+// operands: thread c's K operand comes from bytes [c d/8, (c + 1) d/8) of
+// a code row, a 32-bit word giving two steps (see attn_tc_coord); a V tile
+// mt takes row g from the low nibble and row g + 8 from the high nibble of
+// byte (d/16) g + mt.  Column n = 2q + h: query q, part h (0 high, 1 remainder), so
 // thread (g, c) holds the score of query c for tokens g and g + 8 and
 // accumulates query c.
 
@@ -786,26 +787,60 @@ __device__ __forceinline__ uint32_t attn_tc_lo(uint32_t x) {
 __device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x) { return attn_tc_lo(x >> 4); }
 
 // Physical coordinate of K-index slot `e` (0: 2c, 1: 2c + 1, 2: 2c + 8,
-// 3: 2c + 9) of step s for thread c: word s / 2 of the thread's 32 bytes
-// holds coordinates 2b .. 2b + 7 (b = 32 c + 4 (s / 2)); even steps take the
-// nibbles of bytes b and b + 2, odd steps those of b + 1 and b + 3.
+// 3: 2c + 9) of step s for thread c: word s / 2 of the thread's d/8 bytes
+// holds coordinates 2b .. 2b + 7 (b = c d/8 + 4 (s / 2)); even steps take
+// the nibbles of bytes b and b + 2, odd steps those of b + 1 and b + 3.
+template <int D>
 __device__ __forceinline__ int attn_tc_coord(int c, int s, int e) {
-  const int b = 32 * c + 4 * (s >> 1);
+  const int b = (D / 8) * c + 4 * (s >> 1);
   const int base = 2 * b + 2 * (s & 1) + (e >> 1);  // low (e < 2) or high nibble
   return base + 4 * (e & 1);                        // byte b (+1) or b + 2 (+3)
 }
 
 constexpr int kTcChunk = 16;   // tokens per warp and chunk
 constexpr int kTcStages = 3;   // chunks in flight per warp
-constexpr int kTcRow = 128;    // code bytes per row (d = 256)
-// staged chunk: K rows | V rows (16 x 128 B, 16-byte chunks swizzled by the
-// token index) | K scales | V scales
-constexpr int kTcStage = 2 * kTcChunk * kTcRow + 2 * kTcChunk * 4;
+// staged chunk: K rows | V rows (16 x d/2 bytes; at d = 256 the 16-byte
+// pieces are swizzled by the token index) | K scales | V scales
+template <int D>
+constexpr int tc_stage_bytes() {
+  return 2 * kTcChunk * (D / 2) + 2 * kTcChunk * 4;
+}
+// position of 16-byte piece `ch` of staged row t
+template <int D>
+__device__ __forceinline__ int tc_piece(int t, int ch) {
+  return D == 256 ? (ch ^ (t & 7)) : ch;
+}
+// `N` consecutive 32-bit words of a staged row from byte `b` (4N bytes
+// within one 16-byte piece, or whole pieces)
+template <int D, int N>
+__device__ __forceinline__ void tc_lds_words(uint32_t row, int t, int b, uint32_t (&w)[N]) {
+  if constexpr (N >= 4) {
+#pragma unroll
+    for (int k = 0; k < N / 4; ++k) {
+      const uint4 v = lds128(row + uint32_t((tc_piece<D>(t, b / 16 + k) << 4)));
+      w[4 * k] = v.x;
+      w[4 * k + 1] = v.y;
+      w[4 * k + 2] = v.z;
+      w[4 * k + 3] = v.w;
+    }
+  } else if constexpr (N == 2) {
+    const uint2 v = lds64(row + uint32_t((tc_piece<D>(t, b / 16) << 4) + (b % 16)));
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+    w[0] = lds32(row + uint32_t((tc_piece<D>(t, b / 16) << 4) + (b % 16)));
+  }
+}
 
-template <int ROT>
+template <int D, int ROT>
 __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const AttnArgs a) {
   namespace cg = cooperative_groups;
-  constexpr int D = 256, NQ = 4;
+  constexpr int NQ = 4;
+  constexpr int kTcRow = D / 2;               // code bytes per row
+  constexpr int kTcStage = tc_stage_bytes<D>();
+  constexpr int NS = D / 16;                  // score steps = accumulation tiles
+  constexpr int KW = D / 32;                  // K words per thread and token
+  constexpr int VW = D / 64;                  // V words per thread and token
   using P = Wide<D, ROT>;
   constexpr int W = P::W;
   using AP = AttnPartial<D, NQ>;
@@ -843,11 +878,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
       const int64_t r0 = w_begin + int64_t(ci) * kTcChunk;
       const int rows = n_w - ci * kTcChunk < kTcChunk ? n_w - ci * kTcChunk : kTcChunk;
 #pragma unroll
-      for (int i = lane; i < kTcChunk * (kTcRow / 16); i += 32) {  // 4 pieces per lane
-        const int t = i >> 3, ch = i & 7;
+      for (int i = lane; i < kTcChunk * (kTcRow / 16); i += 32) {  // d / 64 pieces per lane
+        const int t = i / (kTcRow / 16), ch = i % (kTcRow / 16);
         const bool ok = t < rows;
         const int64_t off = ok ? (r0 + t) * kTcRow + ch * 16 : r0 * kTcRow;
-        const uint32_t dst = uint32_t(t * kTcRow + ((ch ^ (t & 7)) << 4));
+        const uint32_t dst = uint32_t(t * kTcRow + (tc_piece<D>(t, ch) << 4));
         cp_async16(st + dst, kbase + off, ok ? 16 : 0);
         cp_async16(st + uint32_t(kTcChunk * kTcRow) + dst, vbase + off, ok ? 16 : 0);
       }
@@ -883,16 +918,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   __syncthreads();
   // B operand of the scores: column g = 2 q + h of step s, rows (slots)
   // 2c, 2c + 1 (qb[s][0]) and 2c + 8, 2c + 9 (qb[s][1])
-  uint32_t qb[16][2];
+  uint32_t qb[NS][2];
   {
     const float* qrow = s_q + (g >> 1) * D;
     const bool rem = g & 1;
 #pragma unroll
-    for (int s = 0; s < 16; ++s)
+    for (int s = 0; s < NS; ++s)
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const float v0 = qrow[attn_tc_coord(c, s, 2 * r)];
-        const float v1 = qrow[attn_tc_coord(c, s, 2 * r + 1)];
+        const float v0 = qrow[attn_tc_coord<D>(c, s, 2 * r)];
+        const float v1 = qrow[attn_tc_coord<D>(c, s, 2 * r + 1)];
         const uint32_t hi = bf16x2_pack(v0, v1);
         const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
         qb[s][r] = rem ? bf16x2_pack(v0 - h0, v1 - h1) : hi;
@@ -900,9 +935,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   }
 
   float m = -INFINITY, l = 0.0f;  // of query c
-  float o[16][4];                 // O^T tiles: coordinates 2 (16 g + mt) (+1), columns 2c, 2c + 1
+  float o[NS][4];  // O^T tiles: coordinates 2 ((d/16) g + mt) (+1), columns 2c, 2c + 1
 #pragma unroll
-  for (int mt = 0; mt < 16; ++mt)
+  for (int mt = 0; mt < NS; ++mt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[mt][i] = 0.0f;
   const uint32_t pw = smem_u32(s_p) + uint32_t(warp * NQ * kTcChunk * 4);
@@ -917,15 +952,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 
     // ---- scores: tokens g and g + 8, query c ----
     float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    {  // bytes [c d/8, (c + 1) d/8) of tokens g and g + 8
+      uint32_t w0[KW], w8[KW];
+      tc_lds_words<D, KW>(kst + uint32_t(g * kTcRow), g, (D / 8) * c, w0);
+      tc_lds_words<D, KW>(kst + uint32_t((g + 8) * kTcRow), g + 8, (D / 8) * c, w8);
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {  // bytes [32c + 16hh, +16) of tokens g and g + 8
-      const uint4 k0 = lds128(kst + uint32_t(g * kTcRow + (((2 * c + hh) ^ (g & 7)) << 4)));
-      const uint4 k8 = lds128(kst + uint32_t((g + 8) * kTcRow + (((2 * c + hh) ^ (g & 7)) << 4)));
-      const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
-      const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w};
-#pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {
-        const int s = 2 * (4 * hh + wi);
+      for (int wi = 0; wi < KW; ++wi) {
+        const int s = 2 * wi;
         mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi]), attn_tc_lo(w8[wi]), attn_tc_hi(w0[wi]),
                           attn_tc_hi(w8[wi]), qb[s][0], qb[s][1]);
         mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi] >> 8), attn_tc_lo(w8[wi] >> 8),
@@ -952,7 +985,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     m = m_new;
     if (__any_sync(kFull, corr != 1.0f)) {
 #pragma unroll
-      for (int mt = 0; mt < 16; ++mt)
+      for (int mt = 0; mt < NS; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[mt][i] *= corr;
     }
@@ -976,15 +1009,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
       }
     }
 
-    // ---- accumulation: V rows 2c, 2c + 1, 2c + 8, 2c + 9, bytes [16g, 16g + 16) ----
+    // ---- accumulation: V rows 2c, 2c + 1, 2c + 8, 2c + 9, bytes [(d/16) g, +d/16) ----
     {
-      auto vrow = [&](int t) { return lds128(vst + uint32_t(t * kTcRow + ((g ^ (t & 7)) << 4))); };
-      const uint4 va = vrow(2 * c), vb = vrow(2 * c + 1);
-      const uint4 vc = vrow(2 * c + 8), vd = vrow(2 * c + 9);
-      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-      const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+      uint32_t wa[VW], wb[VW], wc[VW], wd[VW];
+      tc_lds_words<D, VW>(vst + uint32_t(2 * c * kTcRow), 2 * c, (D / 16) * g, wa);
+      tc_lds_words<D, VW>(vst + uint32_t((2 * c + 1) * kTcRow), 2 * c + 1, (D / 16) * g, wb);
+      tc_lds_words<D, VW>(vst + uint32_t((2 * c + 8) * kTcRow), 2 * c + 8, (D / 16) * g, wc);
+      tc_lds_words<D, VW>(vst + uint32_t((2 * c + 9) * kTcRow), 2 * c + 9, (D / 16) * g, wd);
 #pragma unroll
-      for (int mt = 0; mt < 16; ++mt) {
+      for (int mt = 0; mt < NS; ++mt) {
         const uint32_t sel = uint32_t(mt & 3) | (uint32_t(4 + (mt & 3)) << 8);
         const uint32_t x01 = __byte_perm(wa[mt >> 2], wb[mt >> 2], sel);  // tokens 2c, 2c + 1
         const uint32_t x89 = __byte_perm(wc[mt >> 2], wd[mt >> 2], sel);  // 2c + 8, 2c + 9
@@ -1006,8 +1039,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     mine[2 * c + 1] = l;
   }
 #pragma unroll
-  for (int mt = 0; mt < 16; ++mt) {
-    const int y = 2 * (16 * g + mt);
+  for (int mt = 0; mt < NS; ++mt) {
+    const int y = 2 * ((D / 16) * g + mt);
     mine[2 * NQ + c * D + y] = o[mt][0] + o[mt][1];
     mine[2 * NQ + c * D + y + 1] = o[mt][2] + o[mt][3];
   }
@@ -1015,10 +1048,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 }
 
 // Dynamic shared memory of kvq_attn_tc_kernel.
+template <int D>
 constexpr int attn_tc_smem_bytes() {
-  constexpr int merge = (kAttnWarps * AttnPartial<256, 4>::FLOATS + 2 * 4) * 4;
+  constexpr int merge = (kAttnWarps * AttnPartial<D, 4>::FLOATS + 2 * 4) * 4;
   constexpr int staging =
-      kAttnWarps * kTcStages * kTcStage + 4 * 256 * 4 + kAttnWarps * 4 * kTcChunk * 4;
+      kAttnWarps * kTcStages * tc_stage_bytes<D>() + 4 * D * 4 + kAttnWarps * 4 * kTcChunk * 4;
   return merge > staging ? merge : staging;
 }
 

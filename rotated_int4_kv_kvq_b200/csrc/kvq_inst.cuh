@@ -45,10 +45,15 @@ static __device__ unsigned g_status;
 #ifndef KVQ_ATTN_MAX_CLUSTER
 #define KVQ_ATTN_MAX_CLUSTER 16
 #endif
-// Decode attention at d = g = 256 with 3-4 queries per KV head on the tensor
-// cores (1) or on the FP32 pipes (0).
+// Decode attention with one scale per token (g = d) and at most 4 queries
+// per KV head on the tensor cores (1) or on the FP32 pipes (0)...
 #ifndef KVQ_ATTN_TC
 #define KVQ_ATTN_TC 1
+#endif
+// ... and at d = g = 64 with one query per KV head (instead of the lane-pair
+// kernel).
+#ifndef KVQ_ATTN_TC_64
+#define KVQ_ATTN_TC_64 0
 #endif
 #ifndef KVQ_ATTN_PAIR_TOKENS
 #define KVQ_ATTN_PAIR_TOKENS 8
@@ -401,12 +406,12 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   return attn_launch(kern, cl, smem, L, a);
 }
 
-// d = g = 256 with 3 or 4 queries per KV head: the tensor-core kernel, about
-// 32 tokens per warp and block, one resident block per SM.
-template <int ROT>
+// g = d with at most 4 queries per KV head: the tensor-core kernel, about 32
+// tokens per warp and block, one resident block per SM.
+template <int D, int ROT>
 cudaError_t attn_tc(const AttnLaunch& L) {
-  constexpr auto kern = kvq_attn_tc_kernel<ROT>;
-  constexpr int smem = attn_tc_smem_bytes();
+  constexpr auto kern = kvq_attn_tc_kernel<D, ROT>;
+  constexpr int smem = attn_tc_smem_bytes<D>();
   int max_cluster;
   cudaError_t e = attn_max_cluster<kern>(smem, &max_cluster);
   if (e != cudaSuccess) return e;
@@ -416,18 +421,16 @@ cudaError_t attn_tc(const AttnLaunch& L) {
   const int cl = int(std::max<int64_t>(
       1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
   AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
-             L.nq, 256, L.sm_scale * float(Wide<256, ROT>::KAPPA_D) * kLog2e};
+             L.nq, D, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
   return attn_launch(kern, cl, smem, L, a);
 }
 
 template <int D, int ROT>
 cudaError_t attn_rot(int group, const AttnLaunch& L) {
   if constexpr (D == 64) {
-    if (L.nq == 1) return attn_pair<D, ROT>(group, L);
+    if (L.nq == 1 && !(KVQ_ATTN_TC_64 && group == 64)) return attn_pair<D, ROT>(group, L);
   }
-  if constexpr (D == 256) {
-    if (KVQ_ATTN_TC && group == 256 && L.nq >= 3 && L.nq <= 4) return attn_tc<ROT>(L);
-  }
+  if (KVQ_ATTN_TC && group == D && L.nq <= 4) return attn_tc<D, ROT>(L);
   if (L.nq <= 1) return attn_nq<D, ROT, 1>(group, L);
   if (L.nq <= 2) return attn_nq<D, ROT, 2>(group, L);
   if (L.nq <= 4) return attn_nq<D, ROT, 4>(group, L);
