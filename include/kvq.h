@@ -256,7 +256,8 @@ KVQ_API kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *pack
  * once (R orthonormal: <q, D R^T y> = <R D q, y>), accumulates
  * sum_t p_t y_V,t in the rotated domain and rotates back once per query.
  * Arithmetic is fp32; with one scale per token (group == d) and n_q <= 4
- * the products run on the tensor cores with each query and weight split
+ * (except d = 64 with one query) the products run on the tensor cores,
+ * with each query and weight split
  * into bf16 high and low parts (about 2^-17 relative), below the fp16
  * rounding of the output.
  *
