@@ -506,8 +506,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   const int nblk = int(cluster.num_blocks());
   const int64_t head = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  WideLane<D, ROT> L;
-  L.init(a.signs, lane);
   const int h = lane & 1;
   const int ng = D / a.group;      // scales per token (1 or 2)
   const int sh = ng == 2 ? h : 0;  // the scale of this lane's half
@@ -576,6 +574,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   // the rotated, pre-scaled query: warp 0 rotates it into shared memory,
   // every lane takes its half
   if (warp == 0) {
+    WideLane<D, ROT> L;  // (set up again for the merge: not live through the loop)
+    L.init(a.signs, lane);
     uint32_t xw[C];
     wide_load_words<D, ROT>(a.q + head * D, L, xw);
     float Y[W];
@@ -723,6 +723,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
     mine[0] = mm;
     mine[1] = ls;
   }
+  WideLane<D, ROT> L;
+  L.init(a.signs, lane);
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
@@ -853,8 +855,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   const int64_t head = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  WideLane<D, ROT> L;
-  L.init(a.signs, lane);
 
   // this block's tokens, then this warp's contiguous share (whole chunks)
   const int64_t per = (a.len + nblk - 1) / nblk;
@@ -903,6 +903,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   float* s_q = s_part + kAttnWarps * kTcStages * (kTcStage / 4);
   float* s_p = s_q + NQ * D;  // per warp: weights [4 queries][16 tokens]
   if (warp < NQ) {
+    WideLane<D, ROT> L;  // (set up again for the merge: not live through the loop)
+    L.init(a.signs, lane);
     uint32_t xw[P::C];
     if (warp < a.nq) {
       wide_load_words<D, ROT>(a.q + (head * a.nq + warp) * D, L, xw);
@@ -1044,6 +1046,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     mine[2 * NQ + c * D + y] = o[mt][0] + o[mt][1];
     mine[2 * NQ + c * D + y + 1] = o[mt][2] + o[mt][3];
   }
+  WideLane<D, ROT> L;
+  L.init(a.signs, lane);
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
