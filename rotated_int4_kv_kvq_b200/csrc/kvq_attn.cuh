@@ -779,14 +779,28 @@ __device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
   return d;
 }
 
+// Constants of the nibble conversion kept in registers: with both operands
+// of (x & mask) ^ c immediate the compiler emits two logic ops, with c in a
+// register one three-input op.
+struct TcConsts {
+  uint32_t base, one, off;
+  __device__ __forceinline__ TcConsts() : base(0x43084308u), one(0x3F803F80u), off(0xC308C308u) {
+    asm volatile("" : "+r"(base), "+r"(one), "+r"(off));  // opaque: stay in registers
+  }
+};
+
 // The codes of the low nibbles of bytes 0 and 2 of x as an exact bf16 pair:
 // (x & 0x000F000F) ^ 0x43084308 is 128 + (n ^ 8) = 136 + q, minus 136.
-__device__ __forceinline__ uint32_t attn_tc_lo(uint32_t x) {
-  return bf16x2_fma((x & 0x000F000Fu) ^ 0x43084308u, 0x3F803F80u, 0xC308C308u);
+__device__ __forceinline__ uint32_t attn_tc_lo(uint32_t x, const TcConsts& k) {
+  uint32_t t;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t) : "r"(x), "n"(0x000F000F), "r"(k.base));
+  return bf16x2_fma(t, k.one, k.off);
 }
 // ... of the high nibbles of bytes 0 and 2 (shifted down first: bf16 has
 // only 7 mantissa bits, so a nibble at bits 4-7 would reach the exponent).
-__device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x) { return attn_tc_lo(x >> 4); }
+__device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x, const TcConsts& k) {
+  return attn_tc_lo(x >> 4, k);
+}
 
 // Physical coordinate of K-index slot `e` (0: 2c, 1: 2c + 1, 2: 2c + 8,
 // 3: 2c + 9) of step s for thread c: word s / 2 of the thread's d/8 bytes
@@ -943,6 +957,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[mt][i] = 0.0f;
   const uint32_t pw = smem_u32(s_p) + uint32_t(warp * NQ * kTcChunk * 4);
+  const TcConsts kc;
 
   for (int ci = 0; ci < nchunk; ++ci) {
     cp_async_wait<kTcStages - 2>();
@@ -961,10 +976,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 #pragma unroll
       for (int wi = 0; wi < KW; ++wi) {
         const int s = 2 * wi;
-        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi]), attn_tc_lo(w8[wi]), attn_tc_hi(w0[wi]),
-                          attn_tc_hi(w8[wi]), qb[s][0], qb[s][1]);
-        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi] >> 8), attn_tc_lo(w8[wi] >> 8),
-                          attn_tc_hi(w0[wi] >> 8), attn_tc_hi(w8[wi] >> 8), qb[s + 1][0],
+        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi], kc), attn_tc_lo(w8[wi], kc),
+                          attn_tc_hi(w0[wi], kc), attn_tc_hi(w8[wi], kc), qb[s][0], qb[s][1]);
+        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi] >> 8, kc), attn_tc_lo(w8[wi] >> 8, kc),
+                          attn_tc_hi(w0[wi] >> 8, kc), attn_tc_hi(w8[wi] >> 8, kc), qb[s + 1][0],
                           qb[s + 1][1]);
       }
     }
@@ -1023,8 +1038,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
         const uint32_t sel = uint32_t(mt & 3) | (uint32_t(4 + (mt & 3)) << 8);
         const uint32_t x01 = __byte_perm(wa[mt >> 2], wb[mt >> 2], sel);  // tokens 2c, 2c + 1
         const uint32_t x89 = __byte_perm(wc[mt >> 2], wd[mt >> 2], sel);  // 2c + 8, 2c + 9
-        mma_bf16_m16n8k16(o[mt], attn_tc_lo(x01), attn_tc_hi(x01), attn_tc_lo(x89),
-                          attn_tc_hi(x89), pb[0], pb[1]);
+        mma_bf16_m16n8k16(o[mt], attn_tc_lo(x01, kc), attn_tc_hi(x01, kc), attn_tc_lo(x89, kc),
+                          attn_tc_hi(x89, kc), pb[0], pb[1]);
       }
     }
     __syncwarp();  // the stage and the weights are consumed before they are refilled
