@@ -256,9 +256,11 @@ KVQ_API kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *pack
  * once (R orthonormal: <q, D R^T y> = <R D q, y>), accumulates
  * sum_t p_t y_V,t in the rotated domain and rotates back once per query.
  * Arithmetic is fp32; with one scale per token (group == d) and n_q <= 4
- * (except d = 64 with one query) the products run on the tensor cores,
- * with each query and weight split into bf16 high and low parts (about
- * 2^-17 relative), below the fp16 rounding of the output.
+ * (except d = 64 with one query) the products run on the tensor cores:
+ * scores as exact integer products of the codes with each query in 27-bit
+ * fixed point (error at most 2^-27 of the query's largest coordinate), the
+ * weighted sum of V with each weight split into bf16 high and low parts
+ * (about 2^-17 relative); both below the fp16 rounding of the output.
  *
  *   q         [n_kv_heads][n_q][d] fp16, 16-byte aligned (read)
  *   k_packed, v_packed  [n_kv_heads][cap][d/2] uint8, 16-byte aligned (read)

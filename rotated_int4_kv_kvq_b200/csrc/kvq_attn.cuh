@@ -733,28 +733,43 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
 // One scale per token (g = d), up to 4 queries per KV head (e.g. the
 // Gemma-3-1B shape, d = 256 with 4 queries).  Per warp and chunk of 16
 // tokens the rotated-domain scores and the accumulation run on the tensor
-// cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
-//   scores           S = K Q^T:  M = 16 tokens, N = 8 = 4 queries x (hi, lo),
-//                                K = d rotated coordinates (d / 16 steps);
-//   accumulation     O^T = V^T P'^T:  M = d coordinates (d / 16 tiles), N =
-//                                the same 8 columns, K = the 16 tokens.
-// int4 codes are exact in bf16; each query (and each weight p s_V) is split
-// into a bf16 high part and a bf16 remainder, the two columns of its pair, so
-// products are exact and the two column sums, added at the end, carry ~16
-// significant bits (error ~2^-17 relative, well under the fp16 output's).
-// With one scale per token (g = d) a token's K scale multiplies its score
-// after the dot product and its V scale folds into its weight.
+// cores (mma.sync):
+//   scores           S = K Q^T:  m16n8k32, u8 x s8 -> s32.  M = 16 tokens,
+//                                K = d rotated coordinates (d / 32 steps),
+//                                N = 16 = 4 queries x 4 slices in two
+//                                products of 8 columns;
+//   accumulation     O^T = V^T P'^T:  m16n8k16, bf16 in, fp32 accumulate.
+//                                M = d coordinates (d / 16 tiles), N = 8 = 4
+//                                queries x (hi, lo), K = the 16 tokens.
+// Scores: a code n enters as the byte q + 8 = n ^ 8 (one logic op per four
+// codes) and the accumulator starts at -8 sum_i B[i], so the integer result
+// is the exact product of the signed codes with the query slice B.  Each
+// pre-scaled query is split into fixed point: exponent k with max |q| < 2^k
+// and four signed 7-bit slices, q ~ 2^(k-6) (B_0 + B_1 2^-7 + B_2 2^-14 +
+// B_3 2^-21), error at most 2^(k-28) <= 2^-27 max |q| per coordinate; the
+// four exact integer products combine into the fp32 score.  Accumulation:
+// int4 codes are exact in bf16; each weight p s_V is split into a bf16 high
+// part and a bf16 remainder, the two columns of its pair, so products are
+// exact and the two column sums carry ~16 significant bits (error ~2^-17
+// relative, well under the fp16 output's).  With one scale per token (g = d)
+// a token's K scale multiplies its score after the dot product and its V
+// scale folds into its weight.
 //
-// Fragments (PTX ISA, m16n8k16 with 16-bit inputs; lane = 4 g + c): A holds
-// rows g and g + 8, columns 2c, 2c + 1 and 2c + 8, 2c + 9; B rows (the K
-// index) 2c, 2c + 1, 2c + 8, 2c + 9 of column g; C rows g, g + 8, columns 2c,
-// 2c + 1.  The coordinates of a step may be any permutation applied to both
-// operands: thread c's K operand comes from bytes [c d/8, (c + 1) d/8) of
-// a code row, a 32-bit word giving two steps (see attn_tc_coord); a V tile
-// mt takes row g from the low nibble and row g + 8 from the high nibble of
-// byte (d/16) g + mt.  Column n = 2q + h: query q, part h (0 high, 1 remainder), so
-// thread (g, c) holds the score of query c for tokens g and g + 8 and
-// accumulates query c.
+// Fragments (PTX ISA; lane = 4 g + c).  m16n8k32 with 8-bit inputs: A holds
+// rows g and g + 8, columns 4c .. 4c + 3 and 16 + 4c .. 16 + 4c + 3 (four
+// bytes a register); B rows (the K index) 4c .. 4c + 3 and 16 + 4c .. of
+// column g.  m16n8k16 with 16-bit inputs: A rows g and g + 8, columns 2c,
+// 2c + 1 and 2c + 8, 2c + 9; B rows 2c, 2c + 1, 2c + 8, 2c + 9 of column g.
+// Both: C rows g, g + 8, columns 2c, 2c + 1.  The coordinates of a step may
+// be any permutation applied to both operands: score step s of thread c
+// takes the 32-bit word at byte c d/8 + 4s of tokens g and g + 8, its low
+// nibbles (even coordinates) as K index 4c + i and its high nibbles (odd
+// coordinates) as 16 + 4c + i; a V tile mt takes row g from the low nibble
+// and row g + 8 from the high nibble of byte (d/16) g + mt.  Score column
+// n = 2q + j: query q, slice j (2 + j in the second product); accumulation
+// column n = 2q + h: query q, part h (0 high, 1 remainder).  So thread
+// (g, c) holds the score of query c for tokens g and g + 8 and accumulates
+// query c.
 
 __device__ __forceinline__ void mma_bf16_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1,
                                                   uint32_t a2, uint32_t a3, uint32_t b0,
@@ -783,11 +798,43 @@ __device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
 // of (x & mask) ^ c immediate the compiler emits two logic ops, with c in a
 // register one three-input op.
 struct TcConsts {
-  uint32_t base, one, off;
-  __device__ __forceinline__ TcConsts() : base(0x43084308u), one(0x3F803F80u), off(0xC308C308u) {
-    asm volatile("" : "+r"(base), "+r"(one), "+r"(off));  // opaque: stay in registers
+  uint32_t base, one, off, x8;
+  __device__ __forceinline__ TcConsts()
+      : base(0x43084308u), one(0x3F803F80u), off(0xC308C308u), x8(0x08080808u) {
+    asm volatile("" : "+r"(base), "+r"(one), "+r"(off), "+r"(x8));  // opaque: stay in registers
   }
 };
+
+// The offset codes q + 8 = n ^ 8 of the low nibbles of the four bytes of x,
+// one per byte: (x & 0x0F0F0F0F) ^ 0x08080808.
+__device__ __forceinline__ uint32_t attn_tc_u8(uint32_t x, const TcConsts& k) {
+  uint32_t t;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t) : "r"(x), "n"(0x0F0F0F0F), "r"(k.x8));
+  return t;
+}
+
+// d = a b + c (first step of a chain) and d += a b, u8 x s8 -> s32
+__device__ __forceinline__ void mma_u8s8_m16n8k32(int (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1, int c0, int c1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%10, %11, %10, %11};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1));
+}
+__device__ __forceinline__ void mma_u8s8_m16n8k32(int (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2^n as fp32 for -126 <= n <= 127
+__device__ __forceinline__ float attn_pow2(int n) { return __int_as_float((n + 127) << 23); }
 
 // The codes of the low nibbles of bytes 0 and 2 of x as an exact bf16 pair:
 // (x & 0x000F000F) ^ 0x43084308 is 128 + (n ^ 8) = 136 + q, minus 136.
@@ -800,17 +847,6 @@ __device__ __forceinline__ uint32_t attn_tc_lo(uint32_t x, const TcConsts& k) {
 // only 7 mantissa bits, so a nibble at bits 4-7 would reach the exponent).
 __device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x, const TcConsts& k) {
   return attn_tc_lo(x >> 4, k);
-}
-
-// Physical coordinate of K-index slot `e` (0: 2c, 1: 2c + 1, 2: 2c + 8,
-// 3: 2c + 9) of step s for thread c: word s / 2 of the thread's d/8 bytes
-// holds coordinates 2b .. 2b + 7 (b = c d/8 + 4 (s / 2)); even steps take
-// the nibbles of bytes b and b + 2, odd steps those of b + 1 and b + 3.
-template <int D>
-__device__ __forceinline__ int attn_tc_coord(int c, int s, int e) {
-  const int b = (D / 8) * c + 4 * (s >> 1);
-  const int base = 2 * b + 2 * (s & 1) + (e >> 1);  // low (e < 2) or high nibble
-  return base + 4 * (e & 1);                        // byte b (+1) or b + 2 (+3)
 }
 
 constexpr int kTcChunk = 16;   // tokens per warp and chunk
@@ -854,8 +890,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   constexpr int NQ = 4;
   constexpr int kTcRow = D / 2;               // code bytes per row
   constexpr int kTcStage = tc_stage_bytes<D>();
-  constexpr int NS = D / 16;                  // score steps = accumulation tiles
-  constexpr int KW = D / 32;                  // K words per thread and token
+  constexpr int NS = D / 16;                  // accumulation tiles
+  constexpr int KW = D / 32;                  // score steps = K words per thread and token
   constexpr int VW = D / 64;                  // V words per thread and token
   using P = Wide<D, ROT>;
   constexpr int W = P::W;
@@ -912,10 +948,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 #pragma unroll
   for (int ci = 0; ci < kTcStages - 1; ++ci) issue(ci);
 
-  // rotated, pre-scaled queries (score = <qr, y_K> in log2 units): warp w
-  // rotates query w into shared memory after the staging rings
-  float* s_q = s_part + kAttnWarps * kTcStages * (kTcStage / 4);
-  float* s_p = s_q + NQ * D;  // per warp: weights [4 queries][16 tokens]
+  // rotated, pre-scaled queries (score = <qr, y_K> in log2 units) in fixed
+  // point: warp w rotates query w and splits it into its exponent k and four
+  // 7-bit slices, stored after the staging rings as bytes [j][x & 1][x / 2]
+  // (slice j, coordinate x), with k and the slice sums C_j beside them
+  uint8_t* s_qs = reinterpret_cast<uint8_t*>(s_part + kAttnWarps * kTcStages * (kTcStage / 4));
+  int* s_qk = reinterpret_cast<int*>(s_qs + NQ * 4 * D);  // [query][k, C_0 .. C_3, pad]
+  float* s_p = reinterpret_cast<float*>(s_qk + NQ * 8);    // per warp: weights [4 queries][16 tokens]
   if (warp < NQ) {
     WideLane<D, ROT> L;  // (set up again for the merge: not live through the loop)
     L.init(a.signs, lane);
@@ -928,27 +967,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     }
     float Y[W];
     wide_rotate_fwd<D, ROT>(xw, L, Y);
+    float amax = 0.0f;
 #pragma unroll
-    for (int w = 0; w < W; ++w) s_q[warp * D + L.k2 * W + w] = Y[w] * a.qscale;
+    for (int w = 0; w < W; ++w) {
+      Y[w] *= a.qscale;
+      amax = fmaxf(amax, fabsf(Y[w]));
+    }
+#pragma unroll
+    for (int msk = 1; msk <= 16; msk <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, msk));
+    // max |q| < 2^k (k clamped so that every power of two below is normal)
+    const int k = min(max(int((__float_as_uint(amax) >> 23) & 0xFFu) - 126, -90), 120);
+    const float up = attn_pow2(6 - k);
+    uint8_t* qs = s_qs + warp * 4 * D;
+    int csum[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int x = L.k2 * W + w;
+      float t = Y[w] * up;  // |t| < 64; each step below is exact
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float b = rintf(t);
+        csum[j] += int(b);
+        qs[(2 * j + (x & 1)) * (D / 2) + (x >> 1)] = uint8_t(int(b) & 0xFF);
+        t = (t - b) * 128.0f;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int msk = 1; msk <= 16; msk <<= 1) csum[j] += __shfl_xor_sync(kFull, csum[j], msk);
+    if (lane == 0) {
+      s_qk[warp * 8] = k;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s_qk[warp * 8 + 1 + j] = csum[j];
+    }
   }
   __syncthreads();
-  // B operand of the scores: column g = 2 q + h of step s, rows (slots)
-  // 2c, 2c + 1 (qb[s][0]) and 2c + 8, 2c + 9 (qb[s][1])
-  uint32_t qb[NS][2];
+  // B operands of the scores: column g = 2 q + j of query q = g / 2, slice j
+  // (qa) and 2 + j (qc); step s holds the slices of even coordinates 2m and
+  // odd 2m + 1, m = c d/8 + 4s .. + 3
+  uint32_t qa[KW][2], qc[KW][2];
   {
-    const float* qrow = s_q + (g >> 1) * D;
-    const bool rem = g & 1;
+    const uint8_t* qs = s_qs + (g >> 1) * 4 * D;
+    const int j = g & 1;
 #pragma unroll
-    for (int s = 0; s < NS; ++s)
+    for (int s = 0; s < KW; ++s) {
+      const int m0 = (D / 8) * c + 4 * s;
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const float v0 = qrow[attn_tc_coord<D>(c, s, 2 * r)];
-        const float v1 = qrow[attn_tc_coord<D>(c, s, 2 * r + 1)];
-        const uint32_t hi = bf16x2_pack(v0, v1);
-        const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
-        qb[s][r] = rem ? bf16x2_pack(v0 - h0, v1 - h1) : hi;
+      for (int par = 0; par < 2; ++par) {
+        qa[s][par] = *reinterpret_cast<const uint32_t*>(qs + (2 * j + par) * (D / 2) + m0);
+        qc[s][par] = *reinterpret_cast<const uint32_t*>(qs + (2 * (j + 2) + par) * (D / 2) + m0);
       }
+    }
   }
+  // query c's exponent and the accumulators' start values -8 C_j
+  const float f_hi = attn_pow2(s_qk[c * 8] - 13), f_lo = attn_pow2(s_qk[c * 8] - 27);
+  const int ca0 = -8 * s_qk[c * 8 + 1], ca1 = -8 * s_qk[c * 8 + 2];
+  const int cc0 = -8 * s_qk[c * 8 + 3], cc1 = -8 * s_qk[c * 8 + 4];
 
   float m = -INFINITY, l = 0.0f;  // of query c
   float o[NS][4];  // O^T tiles: coordinates 2 ((d/16) g + mt) (+1), columns 2c, 2c + 1
@@ -968,25 +1043,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     const int rows = n_w - ci * kTcChunk < kTcChunk ? n_w - ci * kTcChunk : kTcChunk;
 
     // ---- scores: tokens g and g + 8, query c ----
-    float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    int sa[4], sc[4];  // slices (0, 1) and (2, 3): exact integer products
     {  // bytes [c d/8, (c + 1) d/8) of tokens g and g + 8
       uint32_t w0[KW], w8[KW];
       tc_lds_words<D, KW>(kst + uint32_t(g * kTcRow), g, (D / 8) * c, w0);
       tc_lds_words<D, KW>(kst + uint32_t((g + 8) * kTcRow), g + 8, (D / 8) * c, w8);
 #pragma unroll
-      for (int wi = 0; wi < KW; ++wi) {
-        const int s = 2 * wi;
-        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi], kc), attn_tc_lo(w8[wi], kc),
-                          attn_tc_hi(w0[wi], kc), attn_tc_hi(w8[wi], kc), qb[s][0], qb[s][1]);
-        mma_bf16_m16n8k16(sacc, attn_tc_lo(w0[wi] >> 8, kc), attn_tc_lo(w8[wi] >> 8, kc),
-                          attn_tc_hi(w0[wi] >> 8, kc), attn_tc_hi(w8[wi] >> 8, kc), qb[s + 1][0],
-                          qb[s + 1][1]);
+      for (int s = 0; s < KW; ++s) {
+        const uint32_t a0 = attn_tc_u8(w0[s], kc), a1 = attn_tc_u8(w8[s], kc);
+        const uint32_t a2 = attn_tc_u8(w0[s] >> 4, kc), a3 = attn_tc_u8(w8[s] >> 4, kc);
+        if (s == 0) {
+          mma_u8s8_m16n8k32(sa, a0, a1, a2, a3, qa[0][0], qa[0][1], ca0, ca1);
+          mma_u8s8_m16n8k32(sc, a0, a1, a2, a3, qc[0][0], qc[0][1], cc0, cc1);
+        } else {
+          mma_u8s8_m16n8k32(sa, a0, a1, a2, a3, qa[s][0], qa[s][1]);
+          mma_u8s8_m16n8k32(sc, a0, a1, a2, a3, qc[s][0], qc[s][1]);
+        }
       }
     }
     const float sk0 = __uint_as_float(lds32(sst + uint32_t(g * 4)));
     const float sk8 = __uint_as_float(lds32(sst + uint32_t((g + 8) * 4)));
-    const float sc0 = g < rows ? (sacc[0] + sacc[1]) * sk0 : -INFINITY;
-    const float sc8 = g + 8 < rows ? (sacc[2] + sacc[3]) * sk8 : -INFINITY;
+    // 2^(k-6) (B_0 + B_1 2^-7 + ...): the slice pairs combine exactly in
+    // integers (|sum| < 2^25), then in fp32
+    const float sc0 =
+        g < rows ? fmaf(float(sc[0] * 128 + sc[1]), f_lo, float(sa[0] * 128 + sa[1]) * f_hi) * sk0
+                 : -INFINITY;
+    const float sc8 =
+        g + 8 < rows ? fmaf(float(sc[2] * 128 + sc[3]), f_lo, float(sa[2] * 128 + sa[3]) * f_hi) * sk8
+                     : -INFINITY;
 
     // ---- online softmax of query c over the chunk (lanes c, c + 4, ...) ----
     float mx = fmaxf(sc0, sc8);
@@ -1070,8 +1154,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
 template <int D>
 constexpr int attn_tc_smem_bytes() {
   constexpr int merge = (kAttnWarps * AttnPartial<D, 4>::FLOATS + 2 * 4) * 4;
-  constexpr int staging =
-      kAttnWarps * kTcStages * tc_stage_bytes<D>() + 4 * D * 4 + kAttnWarps * 4 * kTcChunk * 4;
+  constexpr int staging = kAttnWarps * kTcStages * tc_stage_bytes<D>() + 4 * 4 * D + 4 * 8 * 4 +
+                          kAttnWarps * 4 * kTcChunk * 4;
   return merge > staging ? merge : staging;
 }
 
