@@ -851,6 +851,7 @@ __device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x, const TcConsts& k) {
 
 constexpr int kTcChunk = 16;   // tokens per warp and chunk
 constexpr int kTcStages = 3;   // chunks in flight per warp
+constexpr float kTcSlack = 8.0f;  // log2 units the running maximum may lag
 // staged chunk: K rows | V rows (16 x d/2 bytes; at d = 256 the 16-byte
 // pieces are swizzled by the token index) | K scales | V scales
 template <int D>
@@ -922,26 +923,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   const float* vsc = a.v_scales + head * a.cap;
 
   const uint32_t ring = smem_u32(s_part) + uint32_t(warp * kTcStages * kTcStage);
-  auto issue = [&](int ci) {
+  // copy roles: a chunk's rows are copied in passes of RI rows, lane ->
+  // (row lt + k RI, 16-byte piece lch) in pass k; whole chunks take fixed
+  // per-lane offsets from running source pointers, the last partial chunk
+  // the checked path
+  constexpr int PR = kTcRow / 16;  // pieces per row
+  constexpr int RI = 32 / PR;      // rows per pass
+  constexpr int NPASS = kTcChunk / RI;
+  const int lt = lane / PR, lch = lane % PR;
+  uint32_t dsto[NPASS];
+#pragma unroll
+  for (int k = 0; k < NPASS; ++k) {
+    const int t = lt + k * RI;
+    dsto[k] = uint32_t(t * kTcRow + (tc_piece<D>(t, lch) << 4));
+  }
+  const uint8_t* kcur = kbase + (w_begin + lt) * kTcRow + lch * 16;
+  const uint8_t* vcur = vbase + (w_begin + lt) * kTcRow + lch * 16;
+  const float* scur = (lane < 16 ? ksc : vsc) + w_begin + (lane & 15);
+  auto issue = [&](int ci) {  // called for ci = 0, 1, 2, ... in order
     if (ci < nchunk) {
       const uint32_t st = ring + uint32_t((ci % kTcStages) * kTcStage);
-      const int64_t r0 = w_begin + int64_t(ci) * kTcChunk;
       const int rows = n_w - ci * kTcChunk < kTcChunk ? n_w - ci * kTcChunk : kTcChunk;
+      if (rows == kTcChunk) {
 #pragma unroll
-      for (int i = lane; i < kTcChunk * (kTcRow / 16); i += 32) {  // d / 64 pieces per lane
-        const int t = i / (kTcRow / 16), ch = i % (kTcRow / 16);
-        const bool ok = t < rows;
-        const int64_t off = ok ? (r0 + t) * kTcRow + ch * 16 : r0 * kTcRow;
-        const uint32_t dst = uint32_t(t * kTcRow + (tc_piece<D>(t, ch) << 4));
-        cp_async16(st + dst, kbase + off, ok ? 16 : 0);
-        cp_async16(st + uint32_t(kTcChunk * kTcRow) + dst, vbase + off, ok ? 16 : 0);
-      }
-      {
+        for (int k = 0; k < NPASS; ++k) {
+          cp_async16(st + dsto[k], kcur + k * RI * kTcRow, 16);
+          cp_async16(st + uint32_t(kTcChunk * kTcRow) + dsto[k], vcur + k * RI * kTcRow, 16);
+        }
+        cp_async4(st + uint32_t(2 * kTcChunk * kTcRow + lane * 4), scur, 4);
+      } else {
+        const int64_t r0 = w_begin + int64_t(ci) * kTcChunk;
+#pragma unroll
+        for (int i = lane; i < kTcChunk * PR; i += 32) {  // d / 64 pieces per lane
+          const int t = i / PR, ch = i % PR;
+          const bool ok = t < rows;
+          const int64_t off = ok ? (r0 + t) * kTcRow + ch * 16 : r0 * kTcRow;
+          const uint32_t dst = uint32_t(t * kTcRow + (tc_piece<D>(t, ch) << 4));
+          cp_async16(st + dst, kbase + off, ok ? 16 : 0);
+          cp_async16(st + uint32_t(kTcChunk * kTcRow) + dst, vbase + off, ok ? 16 : 0);
+        }
         const int t = lane & 15;
         const bool ok = t < rows;
         const float* src = (lane < 16 ? ksc : vsc) + (ok ? r0 + t : r0);
         cp_async4(st + uint32_t(2 * kTcChunk * kTcRow + lane * 4), src, ok ? 4 : 0);
       }
+      kcur += kTcChunk * kTcRow;
+      vcur += kTcChunk * kTcRow;
+      scur += kTcChunk;
     }
     cp_async_commit();  // possibly empty: keeps the group count uniform
   };
@@ -1073,23 +1101,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
                      : -INFINITY;
 
     // ---- online softmax of query c over the chunk (lanes c, c + 4, ...) ----
+    // The reference m moves only when the chunk's maximum exceeds it by more
+    // than kTcSlack (weights then stay below 2^kTcSlack), so the accumulators
+    // are rescaled rarely; the merges take any reference.
     float mx = fmaxf(sc0, sc8);
 #pragma unroll
     for (int msk = 4; msk <= 16; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, msk));
-    const float m_new = fmaxf(m, mx);  // finite: the chunk holds a valid token
-    const float corr = exp2f(m - m_new);
-    const float p0 = exp2f(sc0 - m_new), p8 = exp2f(sc8 - m_new);
-    float ps = p0 + p8;
-#pragma unroll
-    for (int msk = 4; msk <= 16; msk <<= 1) ps += __shfl_xor_sync(kFull, ps, msk);
-    l = l * corr + ps;
-    m = m_new;
-    if (__any_sync(kFull, corr != 1.0f)) {
+    if (__any_sync(kFull, mx > m + kTcSlack)) {  // always on the first chunk (m = -inf)
+      const float m_new = mx > m + kTcSlack ? mx : m;  // finite: the chunk holds a valid token
+      const float corr = exp2f(m - m_new);
+      l *= corr;
 #pragma unroll
       for (int mt = 0; mt < NS; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[mt][i] *= corr;
+      m = m_new;
     }
+    const float p0 = exp2f(sc0 - m), p8 = exp2f(sc8 - m);
+    float ps = p0 + p8;
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) ps += __shfl_xor_sync(kFull, ps, msk);
+    l += ps;
     // weights p s_V by (query, token) through shared memory, then the B
     // operand: column g = 2 q + h, tokens 2c, 2c + 1 and 2c + 8, 2c + 9
     const float sv0 = __uint_as_float(lds32(sst + uint32_t((kTcChunk + g) * 4)));

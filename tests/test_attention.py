@@ -22,23 +22,32 @@ def kvq():
     return mod
 
 
-def make_cache(kvq, heads, cap, d, group, rot, signs, seed):
+def make_cache(kvq, heads, cap, d, group, rot, signs, seed, ramp=0.0):
+    """ramp > 0: K rows drift along the all-ones direction (by ramp at the
+    last row) and the queries point along it, so the scores rise through
+    the sequence and the running maximum moves many times."""
     g = torch.Generator(device="cuda").manual_seed(seed)
     out = []
-    for _ in range(2):  # K, V
-        x = (torch.randn((heads * cap, d), generator=g, device="cuda") * 2).half()
+    for kv in range(2):  # K, V
+        x = torch.randn((heads * cap, d), generator=g, device="cuda") * 2
         x[:, 7] *= 15  # an outlier channel
+        if ramp and kv == 0:
+            t = torch.arange(cap, device="cuda", dtype=torch.float32).repeat(heads) / cap
+            x += ramp * t[:, None]
+        x = x.half()
         p, s = kvq.kvq_rot_quant_fwd(x, signs, rot, group)
         out += [p.reshape(heads, cap, -1), s.reshape(heads, cap, -1)]
     q = (torch.randn((heads, 8, d), generator=g, device="cuda")).half()
+    if ramp:
+        q = (q.float() * 0.1 + 1.0).half()
     return out, q
 
 
-def run_case(kvq, d, group, rot, heads, nq, length, sm_scale=None, seed=0):
+def run_case(kvq, d, group, rot, heads, nq, length, sm_scale=None, seed=0, ramp=0.0):
     cap = length + 5
     signs_np = W.make_signs(d)
     signs = torch.from_numpy(signs_np).cuda()
-    (kp, ks, vp, vs), qall = make_cache(kvq, heads, cap, d, group, rot, signs, seed)
+    (kp, ks, vp, vs), qall = make_cache(kvq, heads, cap, d, group, rot, signs, seed, ramp)
     # garbage beyond len
     kp[:, length:] = 0x77
     vp[:, length:] = 0x17
@@ -108,3 +117,14 @@ def test_attention_tensor_core_d256(kvq, rot, heads, nq, length, scale):
     head, flat and sharp softmax, more heads than one block each."""
     run_case(kvq, 256, 256, rot, heads=heads, nq=nq, length=length, sm_scale=scale,
              seed=heads * 7 + nq + length)
+
+
+@pytest.mark.parametrize("d,group,nq", [(256, 256, 4), (128, 128, 3), (64, 64, 2), (64, 64, 1),
+                                        (256, 64, 4)])
+@pytest.mark.parametrize("heads,length", [(1, 4096), (2, 777), (40, 1500)])
+def test_attention_rising_scores(kvq, d, group, nq, heads, length):
+    """Scores that rise through the sequence (by tens of log2 units): the
+    running maximum of every warp moves many times, in steps below and
+    above any slack the kernels allow it."""
+    run_case(kvq, d, group, O.SRFT, heads=heads, nq=nq, length=length, sm_scale=0.5 / d ** 0.5,
+             seed=heads + length + d, ramp=6.0)
