@@ -47,6 +47,13 @@ constexpr int kAttnMaxCluster = 16;  // blocks per KV head at most
 #define KVQ_ATTN_MIXED_UNPACK 1
 #endif
 
+// Lazy online softmax (the lane-pair and tensor-core kernels): a running
+// reference maximum m moves only when a new score exceeds it by more than
+// kAttnSlack (log2 units), so weights 2^(s - m) stay below 2^kAttnSlack and
+// the accumulators are rescaled only then; the warp, block and cluster
+// merges take any reference m with its (l, o).
+constexpr float kAttnSlack = 8.0f;
+
 // Asynchronous global -> shared copies (cp.async); `bytes` < size zero-fills
 // the rest and 0 reads nothing.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int bytes) {
@@ -633,7 +640,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   // one online-softmax update for two scored tokens (s1 = -inf: no second)
   auto update = [&](float s0, float s1, const uint4& vc0, float sv0, const uint4& vc1, float sv1) {
     const float mx = fmaxf(s0, s1);
-    if (mx > m) {  // a new maximum: rescale what has accumulated (m = -inf: zeros)
+    if (mx > m + kAttnSlack) {  // the reference moves: rescale (m = -inf: zeros)
       const float corr = exp2f(m - mx);
       const f2 c2 = mk2(corr, corr);
       l *= corr;
@@ -851,7 +858,6 @@ __device__ __forceinline__ uint32_t attn_tc_hi(uint32_t x, const TcConsts& k) {
 
 constexpr int kTcChunk = 16;   // tokens per warp and chunk
 constexpr int kTcStages = 3;   // chunks in flight per warp
-constexpr float kTcSlack = 8.0f;  // log2 units the running maximum may lag
 // staged chunk: K rows | V rows (16 x d/2 bytes; at d = 256 the 16-byte
 // pieces are swizzled by the token index) | K scales | V scales
 template <int D>
@@ -1101,14 +1107,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
                      : -INFINITY;
 
     // ---- online softmax of query c over the chunk (lanes c, c + 4, ...) ----
-    // The reference m moves only when the chunk's maximum exceeds it by more
-    // than kTcSlack (weights then stay below 2^kTcSlack), so the accumulators
-    // are rescaled rarely; the merges take any reference.
+    // lazy maximum (kAttnSlack)
     float mx = fmaxf(sc0, sc8);
 #pragma unroll
     for (int msk = 4; msk <= 16; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, msk));
-    if (__any_sync(kFull, mx > m + kTcSlack)) {  // always on the first chunk (m = -inf)
-      const float m_new = mx > m + kTcSlack ? mx : m;  // finite: the chunk holds a valid token
+    if (__any_sync(kFull, mx > m + kAttnSlack)) {  // always on the first chunk (m = -inf)
+      const float m_new = mx > m + kAttnSlack ? mx : m;  // finite: the chunk holds a valid token
       const float corr = exp2f(m - m_new);
       l *= corr;
 #pragma unroll
