@@ -347,6 +347,46 @@ cudaError_t attn_max_cluster(int smem, int* out) {
   return cudaSuccess;
 }
 
+// The largest cluster size c <= limit (c >= 1) for which `need` clusters of
+// c blocks are co-resident on the device (one wave), per the occupancy
+// calculator: a cluster must fit in one GPC, so the SMs alone do not decide
+// (e.g. 8 clusters of 16 blocks on 148 SMs take two waves).  Answers are
+// cached per device, kernel and size.
+template <auto Kern, int THREADS = kAttnThreads>
+cudaError_t attn_fit_cluster(int smem, int limit, int64_t need, int* out) {
+  static int maxact[kMaxDevices][kAttnMaxCluster + 1];  // 0: not asked yet
+  static std::mutex mu;
+  int dev;
+  cudaError_t e = current_device(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  int c = std::max(1, std::min(limit, kAttnMaxCluster));
+  for (; c > 1; --c) {
+    if (maxact[dev][c] == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(unsigned(c), 1, 1);
+      q.blockDim = dim3(THREADS, 1, 1);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = unsigned(c);
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      q.attrs = &attr;
+      q.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, Kern, &q) != cudaSuccess) {
+        cudaGetLastError();
+        n = -1;  // not placeable: never chosen
+      }
+      maxact[dev][c] = n > 0 ? n : -1;
+    }
+    if (maxact[dev][c] >= need) break;
+  }
+  *out = c;
+  return cudaSuccess;
+}
+
 // One cluster of `cl` blocks per KV head.
 template <typename... KArgs>
 cudaError_t attn_launch(void (*kern)(KArgs...), int cl, int smem, const AttnLaunch& L,
@@ -380,8 +420,10 @@ cudaError_t attn_pair(int group, const AttnLaunch& L) {
   constexpr int64_t per_block = int64_t(kAttnThreads / 2) * KVQ_ATTN_PAIR_TOKENS;
   const int64_t by_len = (L.len + per_block - 1) / per_block;
   const int64_t by_sms = std::max<int64_t>(1, 2 * int64_t(L.sm_count) / std::max<int64_t>(1, L.n_kv));
-  const int cl = int(std::max<int64_t>(
+  int cl = int(std::max<int64_t>(
       1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  e = attn_fit_cluster<kern>(smem, cl, L.n_kv, &cl);
+  if (e != cudaSuccess) return e;
   AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
              L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
   return attn_launch(kern, cl, smem, L, a);
@@ -399,8 +441,10 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   constexpr int64_t per_block = int64_t(kAttnWarps) * KVQ_ATTN_ROWS_PER_WARP;
   const int64_t by_len = (L.len + per_block - 1) / per_block;
   const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
-  const int cl = int(std::max<int64_t>(
+  int cl = int(std::max<int64_t>(
       1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  e = attn_fit_cluster<kern>(smem, cl, L.n_kv, &cl);
+  if (e != cudaSuccess) return e;
   AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
              L.nq, group, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
   return attn_launch(kern, cl, smem, L, a);
@@ -418,8 +462,10 @@ cudaError_t attn_tc(const AttnLaunch& L) {
   constexpr int64_t per_block = int64_t(kAttnWarps) * 2 * kTcChunk;
   const int64_t by_len = (L.len + per_block - 1) / per_block;
   const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
-  const int cl = int(std::max<int64_t>(
+  int cl = int(std::max<int64_t>(
       1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
+  e = attn_fit_cluster<kern>(smem, cl, L.n_kv, &cl);
+  if (e != cudaSuccess) return e;
   AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
              L.nq, D, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
   return attn_launch(kern, cl, smem, L, a);
