@@ -1049,7 +1049,9 @@ def run_attention_suite(kvq, dev, peak):
     gen = torch.Generator(device=dev).manual_seed(21)
     cases = [("gemma-3-1b step", 26, 1, 4, 256, 256, (256, 1024, 2048, 4096)),
              ("smollm2-1.7b layer", 1, 32, 1, 64, 64, (1024, 4096, 16384)),
+             ("gemma-3-1b layer x 16 sequences", 1, 16, 4, 256, 256, (4096,)),
              ("gemma-3-1b layer x 64 sequences", 1, 64, 4, 256, 256, (4096,)),
+             ("gemma-3-1b layer x 128 sequences", 1, 128, 4, 256, 256, (4096,)),
              ("smollm2-1.7b layer x 16 sequences", 1, 512, 1, 64, 64, (16384,))]
     for name, layers, heads, nq, d, g, lens in cases:
         cap = max(lens)

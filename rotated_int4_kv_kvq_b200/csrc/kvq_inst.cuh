@@ -264,8 +264,8 @@ cudaError_t decode_one(const DecodeLaunch& L) {
                     *L.tmXn, *L.tmQn, *L.tmOn, *L.tmQc, *L.tmOc, a, st);
 }
 
-// Resident 256-thread blocks per SM of a one-warp-per-vector kernel (cached
-// per device).
+// Resident kWideThreads-thread blocks per SM of a one-warp-per-vector kernel
+// (cached per device).
 template <auto Kern>
 cudaError_t wide_occupancy(int* occ_out) {
   static int occ[kMaxDevices];

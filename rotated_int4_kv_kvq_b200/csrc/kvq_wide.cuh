@@ -29,7 +29,9 @@
 namespace kvq {
 
 constexpr float kSqrt2Wide = 1.41421356237309504880f;
-constexpr int kWideThreads = 256;
+// Blocks of 4 warps: a short call (a few hundred rows) spreads over more SMs
+// with at most one warp per scheduler, which shortens each row's latency.
+constexpr int kWideThreads = 128;
 
 // exp(-2 pi i j / 256) for j < 256, rounded once from double.
 struct Tw256 {
