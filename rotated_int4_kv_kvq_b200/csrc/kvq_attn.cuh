@@ -91,6 +91,7 @@ struct AttnArgs {
   int nq;                    // queries per KV head (<= NQ; the rest are padding)
   int group;
   float qscale;              // sm_scale * KAPPA * log2(e)
+  int qgroups;               // tensor-core kernel: blocks of 4 queries per KV head
 };
 
 // Per-warp (or per-block) partial state of one query: running max m (base 2),
@@ -154,7 +155,8 @@ template <int D, int ROT, int NQ>
 __device__ __forceinline__ void attn_merge_store(const AttnArgs& a, float* s_part,
                                                  cooperative_groups::cluster_group& cluster,
                                                  int rank, int nblk, int64_t head, int warp,
-                                                 int lane, const WideLane<D, ROT>& L) {
+                                                 int lane, const WideLane<D, ROT>& L,
+                                                 int q0 = 0, int qn = -1) {
   using P = Wide<D, ROT>;
   constexpr int W = P::W, C = P::C;
   using AP = AttnPartial<D, NQ>;
@@ -241,7 +243,7 @@ __device__ __forceinline__ void attn_merge_store(const AttnArgs& a, float* s_par
     }
   }
   cluster.sync();  // block 0's slot 1 is complete; remote reads done, others may exit
-  if (rank == 0 && warp < a.nq) {
+  if (rank == 0 && warp < (qn < 0 ? a.nq : qn)) {  // queries q0 .. of the KV head
     const int qi = warp;
     const float* fin = s_part + AP::FLOATS + 2 * NQ + qi * D;
     float Y[W];
@@ -249,7 +251,7 @@ __device__ __forceinline__ void attn_merge_store(const AttnArgs& a, float* s_par
     for (int w = 0; w < W; ++w) Y[w] = fin[k2 * W + w] * P::KAPPA;
     uint32_t xo[C];
     wide_rotate_inv<D, ROT>(Y, L, xo);
-    wide_store_words<D, ROT>(a.out + (head * a.nq + qi) * D, L, xo);
+    wide_store_words<D, ROT>(a.out + (head * a.nq + q0 + qi) * D, L, xo);
   }
 }
 
@@ -891,8 +893,12 @@ __device__ __forceinline__ void tc_lds_words(uint32_t row, int t, int b, uint32_
   }
 }
 
-template <int D, int ROT>
-__global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const AttnArgs a) {
+// QG: more than 4 queries per KV head, one grid row per (head, group of 4
+// queries); else one grid row per head.  (Two resident blocks per SM up to
+// d = 128: at most 128 registers.)
+template <int D, int ROT, bool QG>
+__global__ void __launch_bounds__(kAttnThreads, D <= 128 ? 2 : 1)
+    kvq_attn_tc_kernel(const AttnArgs a) {
   namespace cg = cooperative_groups;
   constexpr int NQ = 4;
   constexpr int kTcRow = D / 2;               // code bytes per row
@@ -909,7 +915,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = int(cluster.block_rank());
   const int nblk = int(cluster.num_blocks());
-  const int64_t head = blockIdx.y;
+  // grid row = KV head, or (KV head, group of 4 queries): queries q0 .. q0 + qn - 1
+  const int64_t head = QG ? blockIdx.y / a.qgroups : blockIdx.y;
+  const int q0 = QG ? int(blockIdx.y - head * a.qgroups) * NQ : 0;
+  const int qn = QG ? (a.nq - q0 < NQ ? a.nq - q0 : NQ) : a.nq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
 
@@ -993,8 +1002,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
     WideLane<D, ROT> L;  // (set up again for the merge: not live through the loop)
     L.init(a.signs, lane);
     uint32_t xw[P::C];
-    if (warp < a.nq) {
-      wide_load_words<D, ROT>(a.q + (head * a.nq + warp) * D, L, xw);
+    if (warp < qn) {
+      wide_load_words<D, ROT>(a.q + (head * a.nq + q0 + warp) * D, L, xw);
     } else {
 #pragma unroll
       for (int j = 0; j < P::C; ++j) xw[j] = 0u;
@@ -1183,7 +1192,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_tc_kernel(const Attn
   }
   WideLane<D, ROT> L;
   L.init(a.signs, lane);
-  attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
+  if constexpr (QG) {
+    attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L, q0, qn);
+  } else {
+    attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
+  }
 }
 
 // Dynamic shared memory of kvq_attn_tc_kernel.

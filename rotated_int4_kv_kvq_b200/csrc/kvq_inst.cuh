@@ -390,9 +390,9 @@ cudaError_t attn_fit_cluster(int smem, int limit, int64_t need, int* out) {
 // One cluster of `cl` blocks per KV head.
 template <typename... KArgs>
 cudaError_t attn_launch(void (*kern)(KArgs...), int cl, int smem, const AttnLaunch& L,
-                        const AttnArgs& a) {
+                        const AttnArgs& a, int64_t grid_y = 0) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(cl), unsigned(L.n_kv), 1);
+  cfg.gridDim = dim3(unsigned(cl), unsigned(grid_y > 0 ? grid_y : L.n_kv), 1);
   cfg.blockDim = dim3(kAttnThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = L.stream;
@@ -450,25 +450,31 @@ cudaError_t attn_nq(int group, const AttnLaunch& L) {
   return attn_launch(kern, cl, smem, L, a);
 }
 
-// g = d with at most 4 queries per KV head: the tensor-core kernel, about 32
-// tokens per warp and block, one resident block per SM.
-template <int D, int ROT>
+// g = d with at most 8 queries per KV head: the tensor-core kernel, about 32
+// tokens per warp and block, one resident block per SM.  Each grid row is a
+// (KV head, group of 4 queries) pair; the two groups of a head run side by
+// side, so the second one reads the head's codes mostly from L2.
+template <int D, int ROT, bool QG>
 cudaError_t attn_tc(const AttnLaunch& L) {
-  constexpr auto kern = kvq_attn_tc_kernel<D, ROT>;
+  constexpr auto kern = kvq_attn_tc_kernel<D, ROT, QG>;
   constexpr int smem = attn_tc_smem_bytes<D>();
   int max_cluster;
   cudaError_t e = attn_max_cluster<kern>(smem, &max_cluster);
   if (e != cudaSuccess) return e;
+  const int qgroups = (L.nq + 3) / 4;
+  const int64_t rows = L.n_kv * qgroups;
   constexpr int64_t per_block = int64_t(kAttnWarps) * 2 * kTcChunk;
   const int64_t by_len = (L.len + per_block - 1) / per_block;
-  const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, L.n_kv));
+  const int64_t by_sms = std::max<int64_t>(1, L.sm_count / std::max<int64_t>(1, rows));
   int cl = int(std::max<int64_t>(
       1, std::min<int64_t>(max_cluster, std::min<int64_t>(by_len, by_sms))));
-  e = attn_fit_cluster<kern>(smem, cl, L.n_kv, &cl);
+  e = attn_fit_cluster<kern>(smem, cl, rows, &cl);
   if (e != cudaSuccess) return e;
-  AttnArgs a{L.q, L.k_packed, L.k_scales, L.v_packed, L.v_scales, L.out, L.signs, L.cap, L.len,
-             L.nq, D, L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e};
-  return attn_launch(kern, cl, smem, L, a);
+  AttnArgs a{L.q,      L.k_packed, L.k_scales, L.v_packed,
+             L.v_scales, L.out,    L.signs,    L.cap,
+             L.len,    L.nq,       D,          L.sm_scale * float(Wide<D, ROT>::KAPPA_D) * kLog2e,
+             qgroups};
+  return attn_launch(kern, cl, smem, L, a, rows);
 }
 
 template <int D, int ROT>
@@ -476,7 +482,9 @@ cudaError_t attn_rot(int group, const AttnLaunch& L) {
   if constexpr (D == 64) {
     if (L.nq == 1 && !(KVQ_ATTN_TC_64 && group == 64)) return attn_pair<D, ROT>(group, L);
   }
-  if (KVQ_ATTN_TC && group == D && L.nq <= 4) return attn_tc<D, ROT>(L);
+  if (KVQ_ATTN_TC && group == D && L.nq <= 4) return attn_tc<D, ROT, false>(L);
+  if (KVQ_ATTN_TC && group == D && L.n_kv <= 32767)  // grid rows <= 65535
+    return attn_tc<D, ROT, true>(L);
   if (L.nq <= 1) return attn_nq<D, ROT, 1>(group, L);
   if (L.nq <= 2) return attn_nq<D, ROT, 2>(group, L);
   if (L.nq <= 4) return attn_nq<D, ROT, 4>(group, L);

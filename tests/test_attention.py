@@ -128,3 +128,16 @@ def test_attention_rising_scores(kvq, d, group, nq, heads, length):
     above any slack the kernels allow it."""
     run_case(kvq, d, group, O.SRFT, heads=heads, nq=nq, length=length, sm_scale=0.5 / d ** 0.5,
              seed=heads + length + d, ramp=6.0)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("rot", [O.SRFT, O.SRHT])
+@pytest.mark.parametrize("heads,nq,length,scale", [(1, 5, 1, None), (2, 8, 17, None), (3, 6, 700, 2.0),
+                                                   (1, 8, 4096, None), (40, 7, 333, None),
+                                                   (2, 8, 1000, 0.0), (100, 8, 64, None)])
+def test_attention_tensor_core_query_groups(kvq, d, rot, heads, nq, length, scale):
+    """g = d with 5-8 queries per KV head: the tensor-core kernel in two
+    groups of 4 queries per head (the second group partly padding for 5-7),
+    single and many heads, ragged lengths, flat and sharp softmax."""
+    run_case(kvq, d, d, rot, heads=heads, nq=nq, length=length, sm_scale=scale,
+             seed=heads * 11 + nq + length + d)
