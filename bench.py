@@ -1052,7 +1052,8 @@ def run_attention_suite(kvq, dev, peak):
              ("gemma-3-1b layer x 16 sequences", 1, 16, 4, 256, 256, (4096,)),
              ("gemma-3-1b layer x 64 sequences", 1, 64, 4, 256, 256, (4096,)),
              ("gemma-3-1b layer x 128 sequences", 1, 128, 4, 256, 256, (4096,)),
-             ("smollm2-1.7b layer x 16 sequences", 1, 512, 1, 64, 64, (16384,))]
+             ("smollm2-1.7b layer x 16 sequences", 1, 512, 1, 64, 64, (16384,)),
+             ("8 queries per kv head, d = 128, x 16 sequences", 1, 128, 8, 128, 128, (4096,))]
     for name, layers, heads, nq, d, g, lens in cases:
         cap = max(lens)
         signs = torch.from_numpy(W.make_signs(d)).to(dev)
