@@ -737,10 +737,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) kvq_attn_pair_kernel(const At
   attn_merge_store<D, ROT, NQ>(a, s_part, cluster, rank, nblk, head, warp, lane, L);
 }
 
-// ----------------------------- tensor-core decode attention (g = d, up to 4 queries) ---
+// ----------------------------- tensor-core decode attention (g = d, up to 8 queries) ---
 //
-// One scale per token (g = d), up to 4 queries per KV head (e.g. the
-// Gemma-3-1B shape, d = 256 with 4 queries).  Per warp and chunk of 16
+// One scale per token (g = d), up to 4 queries per block and up to 8 per KV
+// head (e.g. the Gemma-3-1B shape, d = 256 with 4 queries).  Per warp and chunk of 16
 // tokens the rotated-domain scores and the accumulation run on the tensor
 // cores (mma.sync):
 //   scores           S = K Q^T:  m16n8k32, u8 x s8 -> s32.  M = 16 tokens,
