@@ -255,9 +255,9 @@ KVQ_API kvq_status kvq_decode_step_windowed(const uint16_t *x_new, uint8_t *pack
  * Only codes and scales are read from memory: the kernel rotates each query
  * once (R orthonormal: <q, D R^T y> = <R D q, y>), accumulates
  * sum_t p_t y_V,t in the rotated domain and rotates back once per query.
- * Arithmetic is fp32; with one scale per token (group == d) (except d = 64
- * with one query) the products run on the tensor cores, in groups of up to
- * 4 queries:
+ * Arithmetic is fp32.  With one scale per token (group == d) the products
+ * run on the tensor cores, up to 4 queries per thread block (except d = 64
+ * with one query, and more than 4 queries over more than 32,767 KV heads):
  * scores as exact integer products of the codes with each query in 27-bit
  * fixed point (error at most 2^-27 of the query's largest coordinate), the
  * weighted sum of V with each weight split into bf16 high and low parts
