@@ -87,9 +87,16 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+# torch's query of a device's current raw stream handle; building a
+# torch.cuda.Stream object per call costs ~2 us, the raw query ~0.1 us.
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream, dev: torch.device) -> int | None:
     """Raw handle of `stream`; None means the current stream of `dev`."""
     if stream is None:
+        if _raw_current_stream is not None and dev.index is not None:
+            return _raw_current_stream(dev.index)
         stream = torch.cuda.current_stream(dev)
     return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
 
@@ -125,7 +132,7 @@ def _check(t: torch.Tensor, name: str, dtype, shape):
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if tuple(t.shape) != tuple(shape):
+    if t.shape != tuple(shape):  # torch.Size compares as a tuple
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
