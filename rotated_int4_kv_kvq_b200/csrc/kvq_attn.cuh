@@ -295,12 +295,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
   constexpr int CB = attn_chunk_bytes<D>();
   const uint32_t ring = smem_u32(s_part) + uint32_t(warp * kAttnStages * CB);
   const int nchunk = int((n_w + kAttnChunk - 1) / kAttnChunk);
-  auto issue = [&](int c) {
+  // whole chunks: every lane copies fixed pieces from running source
+  // pointers (piece i = lane + 32k of the code tile is row i / PR, 16-byte
+  // column i % PR), and the chunk's scales as one contiguous run (16-byte
+  // pieces where both scale bases allow it); the last, partial chunk takes
+  // the checked path
+  constexpr int PR = QROW / 16;
+  const uint8_t* kcur = kbase + (w_begin + lane / PR) * QROW + (lane % PR) * 16;
+  const uint8_t* vcur = vbase + (w_begin + lane / PR) * QROW + (lane % PR) * 16;
+  const float* kscur = ksc + w_begin * ng;
+  const float* vscur = vsc + w_begin * ng;
+  const bool sc16 =
+      ((reinterpret_cast<uintptr_t>(kscur) | reinterpret_cast<uintptr_t>(vscur)) & 15u) == 0;
+  auto issue = [&](int c) {  // called for c = 0, 1, 2, ... in order
     if (c < nchunk) {
       const uint32_t st = ring + uint32_t((c % kAttnStages) * CB);
       const int64_t r0 = w_begin + int64_t(c) * kAttnChunk;
       const int rows = int(w_end - r0 < kAttnChunk ? w_end - r0 : kAttnChunk);
       constexpr int PIECES = kAttnChunk * QROW / 16;  // 16-byte pieces per code tile
+      const uint32_t sk = st + uint32_t(2 * kAttnChunk * QROW);
+      const uint32_t sv = sk + uint32_t(kAttnChunk * (D / 32) * 4);
+      if (rows == kAttnChunk) {
+#pragma unroll
+        for (int k = 0; k < PIECES / 32; ++k) {
+          cp_async16(st + uint32_t((lane + 32 * k) * 16), kcur + k * 512, 16);
+          cp_async16(st + uint32_t(kAttnChunk * QROW + (lane + 32 * k) * 16), vcur + k * 512, 16);
+        }
+        if (sc16) {
+          for (int i = lane; i < 8 * ng; i += 32) {  // 32 ng floats in 16-byte pieces
+            cp_async16(sk + uint32_t(i * 16), kscur + 4 * i, 16);
+            cp_async16(sv + uint32_t(i * 16), vscur + 4 * i, 16);
+          }
+        } else {
+          for (int i = lane; i < kAttnChunk * ng; i += 32) {
+            cp_async4(sk + uint32_t(i * 4), kscur + i, 4);
+            cp_async4(sv + uint32_t(i * 4), vscur + i, 4);
+          }
+        }
+        kcur += kAttnChunk * QROW;
+        vcur += kAttnChunk * QROW;
+        kscur += kAttnChunk * ng;
+        vscur += kAttnChunk * ng;
+        cp_async_commit();
+        return;
+      }
 #pragma unroll
       for (int i = lane; i < PIECES; i += 32) {
         const int row = i / (QROW / 16);
@@ -309,8 +347,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) kvq_attn_kernel(const AttnArg
         cp_async16(st + uint32_t(i * 16), kbase + off, ok ? 16 : 0);
         cp_async16(st + uint32_t(kAttnChunk * QROW + i * 16), vbase + off, ok ? 16 : 0);
       }
-      const uint32_t sk = st + uint32_t(2 * kAttnChunk * QROW);
-      const uint32_t sv = sk + uint32_t(kAttnChunk * (D / 32) * 4);
       for (int i = lane; i < kAttnChunk * ng; i += 32) {
         const int row = i / ng;
         const bool ok = row < rows;
